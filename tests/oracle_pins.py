@@ -1,0 +1,353 @@
+"""Pins for the CPU oracle: checks against things other than the oracle itself.
+
+Each pin takes an ``oracle.Oracle`` and raises AssertionError when the oracle
+disagrees with brute force, a closed form, an invariant, a hand-worked example
+(tests/golden/hand_example.json) or a library routine.  ``test_oracle_pins``
+runs them on the committed oracle; ``test_oracle_mutants`` runs them on
+deliberately broken copies of it and expects at least one to fail each time.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_example.json")
+
+
+def _rng(seed=0):
+    return np.random.default_rng(seed)
+
+
+def _tie_free_logits(n, e, seed=0):
+    # distinct values per row: a random permutation of a spread grid plus noise
+    r = _rng(seed)
+    base = np.stack([r.permutation(e) for _ in range(n)]).astype(np.float64)
+    return (base * 0.37 + r.uniform(-0.1, 0.1, (n, e))).astype(np.float32)
+
+
+# ------------------------------------------------------------------ route
+def pin_route_bruteforce(o):
+    """Top-k = first k of the full sort of (-logit, id): brute force, with ties."""
+    r = _rng(1)
+    for (n, e, k) in [(37, 8, 2), (20, 16, 5), (9, 6, 6), (12, 32, 1)]:
+        # coarse grid -> many exact ties
+        logits = r.integers(-3, 4, size=(n, e)).astype(np.float32) * 0.5
+        idx, _ = o.route(logits, k)
+        for t in range(n):
+            ref = sorted(range(e), key=lambda ex: (-float(logits[t, ex]), ex))[:k]
+            assert list(idx[t]) == ref, (n, e, k, t, list(idx[t]), ref)
+
+
+def pin_route_torch_topk(o):
+    """On tie-free rows the selection equals torch.topk (a library routine)."""
+    for (n, e, k) in [(64, 8, 2), (50, 256, 8), (40, 128, 4)]:
+        logits = _tie_free_logits(n, e, seed=n + e)
+        idx, _ = o.route(logits, k)
+        ref = torch.topk(torch.from_numpy(logits), k, dim=1, sorted=True).indices.numpy()
+        assert np.array_equal(idx, ref)
+
+
+def pin_route_special_cases(o):
+    """All-equal logits pick experts 0..k-1 with weight 1/k; k=1 gives weight 1;
+    k=E returns every expert in descending logit order."""
+    logits = np.full((3, 8), 0.25, np.float32)
+    idx, w = o.route(logits, 3)
+    assert np.array_equal(idx, np.tile(np.arange(3), (3, 1)))
+    assert np.all(w == np.float32(1.0 / 3.0))
+    logits = _tie_free_logits(10, 16, seed=5)
+    idx, w = o.route(logits, 1)
+    assert np.array_equal(idx[:, 0], logits.argmax(1)) and np.all(w == 1.0)
+    idx, w = o.route(logits, 16)
+    assert np.array_equal(idx, np.argsort(-logits, axis=1, kind="stable"))
+
+
+def pin_route_weights_closed_form(o):
+    """k=2: w0 = 1/(1+exp(L1-L0)) (the logistic form); general k: softmax of
+    the selected logits via scipy; weights sum to 1 and do not increase in j."""
+    from scipy.special import softmax
+    logits = _tie_free_logits(40, 8, seed=7) * 3.0
+    idx, w = o.route(logits, 2)
+    for t in range(40):
+        l0, l1 = float(logits[t, idx[t, 0]]), float(logits[t, idx[t, 1]])
+        ref0 = 1.0 / (1.0 + math.exp(l1 - l0))
+        assert abs(float(w[t, 0]) - ref0) <= 2 ** -24 * ref0 * 2
+        assert abs(float(w[t, 1]) - (1.0 - ref0)) <= 2 ** -24 * 2
+    logits = _tie_free_logits(30, 64, seed=8) * 2.0
+    idx, w = o.route(logits, 6)
+    sel = np.take_along_axis(logits.astype(np.float64), idx.astype(np.int64), axis=1)
+    ref = softmax(sel, axis=1)
+    assert np.allclose(w, ref, rtol=2 ** -22, atol=0)
+    assert np.allclose(w.astype(np.float64).sum(1), 1.0, atol=1e-6)
+    assert np.all(np.diff(w, axis=1) <= 0)
+
+
+# ------------------------------------------------------------------ layout
+def pin_counts_bincount(o):
+    """counts = numpy bincount of the flattened picks; they sum to N*k."""
+    logits = _tie_free_logits(100, 16, seed=9)
+    idx, _ = o.route(logits, 4)
+    c = o.counts(idx, 16)
+    assert np.array_equal(c, np.bincount(idx.ravel(), minlength=16))
+    assert c.sum() == 100 * 4
+
+
+def pin_offsets(o):
+    """R=1: exclusive prefix sum (numpy cumsum).  R>1: each rank's experts
+    start at the fixed base r*N*min(k,E/R) and are packed inside it."""
+    r = _rng(3)
+    for (n, e, k, ranks) in [(50, 16, 4, 1), (50, 16, 4, 4), (33, 8, 4, 4), (7, 12, 3, 3)]:
+        idx = np.stack([r.permutation(e)[:k] for _ in range(n)]).astype(np.int32)
+        c = o.counts(idx, e)
+        off = o.offsets(n, e, k, ranks, c)
+        per = e // ranks
+        c_r = n * min(k, per)
+        assert o.region_rows(n, e, k, ranks) == c_r
+        assert off[e] == ranks * c_r
+        for rank in range(ranks):
+            lo = rank * per
+            seg = off[lo:lo + per]
+            ref = rank * c_r + np.concatenate([[0], np.cumsum(c[lo:lo + per])[:-1]])
+            assert np.array_equal(seg, ref)
+            assert seg[-1] + c[lo + per - 1] <= (rank + 1) * c_r
+    # worst case: every token sends min(k, E/R) rows to rank 0 -> exactly fills it
+    n, e, k, ranks = 5, 8, 4, 4
+    idx = np.tile(np.array([0, 1, 2, 3], np.int32), (n, 1))
+    c = o.counts(idx, e)
+    off = o.offsets(n, e, k, ranks, c)
+    assert off[1] + c[1] == o.region_rows(n, e, k, ranks) == off[2]
+
+
+def pin_slots_stable_sort(o):
+    """R=1: slot order is the stable argsort of the flattened picks (the sorted
+    gather path); any R: brute-force count of earlier tokens per expert, the
+    map is a bijection onto the filled slots and src_of inverts slot_of."""
+    r = _rng(4)
+    for (n, e, k, ranks) in [(60, 8, 2, 1), (60, 8, 2, 2), (45, 16, 4, 4), (10, 4, 4, 2)]:
+        idx = np.stack([r.permutation(e)[:k] for _ in range(n)]).astype(np.int32)
+        c = o.counts(idx, e)
+        off = o.offsets(n, e, k, ranks, c)
+        slot_of, src_of = o.slots(idx, off, e)
+        if ranks == 1:
+            order = np.argsort(idx.ravel(), kind="stable")
+            assert np.array_equal(src_of[: n * k], order)
+        for t in range(n):
+            for j in range(k):
+                ex = idx[t, j]
+                earlier = sum(1 for t2 in range(t) if ex in idx[t2])
+                assert slot_of[t, j] == off[ex] + earlier
+        flat = slot_of.ravel()
+        assert len(np.unique(flat)) == n * k
+        assert np.array_equal(src_of[flat], np.arange(n * k))
+        filled = np.zeros(src_of.size, bool)
+        filled[flat] = True
+        assert np.all(src_of[~filled] == -1)
+
+
+def pin_dispatch_repeat_interleave(o):
+    """recv gathered at slot_of equals x.repeat_interleave(k) (the unsorted
+    path); every source row appears exactly k times; unfilled rows are zero."""
+    r = _rng(5)
+    n, e, k, ranks, d = 40, 8, 3, 2, 24
+    idx = np.stack([r.permutation(e)[:k] for _ in range(n)]).astype(np.int32)
+    x = r.standard_normal((n, d)).astype(np.float32)
+    c = o.counts(idx, e)
+    off = o.offsets(n, e, k, ranks, c)
+    slot_of, src_of = o.slots(idx, off, e)
+    recv = o.scatter_rows(x, slot_of, int(off[e]))
+    ref = torch.from_numpy(x).repeat_interleave(k, dim=0).numpy()
+    assert np.array_equal(recv[slot_of.ravel()], ref)
+    filled = src_of >= 0
+    assert np.all(recv[~filled] == 0)
+    # bytes too: a bf16 and an fp8 payload travel unchanged
+    xb = r.integers(0, 2 ** 16, size=(n, d), dtype=np.uint16)
+    rb = o.scatter_rows(xb, slot_of, int(off[e]))
+    assert np.array_equal(rb[slot_of.ravel()], np.repeat(xb, k, axis=0))
+
+
+# ------------------------------------------------------------------ numbers
+def pin_e4m3_decode(o):
+    """All 256 e4m3 codes decode as torch.float8_e4m3fn does (library)."""
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = np.array([o.e4m3_to_float(c) for c in range(256)])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+
+
+def pin_bf16_rounding(o):
+    """Round-to-nearest-even to bf16: hand cases (ties, subnormals, overflow)
+    and agreement with torch's float32 -> bfloat16 cast on random floats."""
+    assert o.bf16_from_float(1.0) == 0x3F80
+    assert o.bf16_from_float(1.0 + 2 ** -8) == 0x3F80          # tie -> even
+    assert o.bf16_from_float(1.0 + 3 * 2 ** -8) == 0x3F82      # tie -> even (up)
+    assert o.bf16_from_float(1.0 + 2 ** -8 + 2 ** -30) == 0x3F81
+    assert o.bf16_from_float(-2.0) == 0xC000
+    assert o.bf16_from_float(2 ** -133) == 0x0001              # smallest subnormal
+    assert o.bf16_from_float(2 ** -134) == 0x0000              # tie -> even (zero)
+    assert o.bf16_from_float(1.5 * 2 ** -133) == 0x0002        # tie -> even (up)
+    assert o.bf16_from_float(3.0e38) == 0x7F62
+    assert o.bf16_from_float(3.4e38) == 0x7F80                 # overflow -> inf
+    assert o.bf16_from_float(float("inf")) == 0x7F80
+    r = _rng(6)
+    f = np.concatenate([r.standard_normal(4000) * 10.0 ** r.integers(-30, 30, 4000),
+                        r.standard_normal(1000)]).astype(np.float32)
+    ref = torch.from_numpy(f).to(torch.bfloat16).view(torch.int16).numpy().astype(np.uint16)
+    got = np.array([o.bf16_from_float(float(v)) for v in f], np.uint16)
+    assert np.array_equal(got, ref)
+    # decode is exact widening
+    bits = r.integers(0, 0x7F80, 500).astype(np.uint16)
+    ref = torch.from_numpy(bits.astype(np.int16)).view(torch.bfloat16).double().numpy()
+    got = np.array([o.bf16_to_float(int(b)) for b in bits])
+    assert np.array_equal(got, ref)
+
+
+def pin_dequant(o):
+    """Identity expert on FP8 rows: with power-of-two scales code*scale is exact,
+    so it equals torch's e4m3 -> float -> bf16 cast bit for bit; with general
+    scales it is within half a bf16 ulp of the exact double product."""
+    r = _rng(7)
+    t, d, blk = 6, 256, 128
+    q = r.integers(0, 256, size=(t, d), dtype=np.uint8)
+    q[(q & 0x7F) == 0x7F] = 0x11           # no NaN codes
+    scale = (2.0 ** r.integers(-8, 8, size=(t, d // blk))).astype(np.float32)
+    rows = np.arange(t, dtype=np.int32)
+    y = o.dequant_rows(rows, q, scale, blk)
+    qf = torch.from_numpy(q).view(torch.float8_e4m3fn).float()
+    ref = (qf * torch.from_numpy(np.repeat(scale, blk, axis=1))).to(torch.bfloat16)
+    assert np.array_equal(y, ref.view(torch.int16).numpy().astype(np.uint16))
+    scale = r.uniform(0.001, 3.0, size=(t, d // blk)).astype(np.float32)
+    y = o.dequant_rows(rows, q, scale, blk)
+    exact = (qf.double() * torch.from_numpy(np.repeat(scale, blk, axis=1)).double()).numpy()
+    yv = o.to_float(y, "bf16")
+    ulp = np.where(exact != 0, 2.0 ** (np.floor(np.log2(np.abs(exact) + 1e-300)) - 7), 0)
+    assert np.all(np.abs(yv - exact) <= 0.5 * ulp + 1e-300)
+    # rows not listed stay untouched (zero)
+    y2 = o.dequant_rows(np.array([1], np.int32), q, scale, blk)
+    assert np.all(y2[0] == 0) and np.array_equal(y2[1], y[1])
+
+
+def _bf16_bits(a: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(torch.bfloat16) \
+        .view(torch.int16).numpy().astype(np.uint16)
+
+
+def _bf16_val(b: np.ndarray) -> np.ndarray:
+    return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def pin_swiglu_dense(o):
+    """One expert holding every row reduces to a dense SwiGLU MLP, computed
+    here with numpy float64 matmuls (library); zero weights give zero output;
+    the expert id selects the weights."""
+    r = _rng(8)
+    rows_n, d, inter, e = 9, 64, 48, 3
+    x = _bf16_bits(r.standard_normal((rows_n, d)))
+    wgu = _bf16_bits(r.standard_normal((e, 2 * inter, d)) * 0.1)
+    wd = _bf16_bits(r.standard_normal((e, d, inter)) * 0.1)
+    rows = np.arange(rows_n, dtype=np.int32)
+    for ex in range(e):
+        y, h = o.swiglu_rows(rows, np.full(rows_n, ex, np.int32), x, wgu, wd, want_h=True)
+        xv = _bf16_val(x)
+        g = xv @ _bf16_val(wgu[ex, :inter]).T
+        u = xv @ _bf16_val(wgu[ex, inter:]).T
+        h_ref = g / (1.0 + np.exp(-g)) * u
+        hv = _bf16_val(h)
+        assert np.all(np.abs(hv - h_ref) <= np.abs(h_ref) * 2 ** -8 + 1e-30)
+        y_ref = hv @ _bf16_val(wd[ex]).T
+        yv = _bf16_val(y)
+        assert np.all(np.abs(yv - y_ref) <= np.abs(y_ref) * 2 ** -8 + 1e-30)
+    # mixed experts per row pick the right weights
+    re = (np.arange(rows_n) % e).astype(np.int32)
+    ymix = o.swiglu_rows(rows, re, x, wgu, wd)
+    for i in range(rows_n):
+        yi = o.swiglu_rows(np.array([i], np.int32), np.array([re[i]], np.int32), x, wgu, wd)
+        assert np.array_equal(ymix[i], yi[i])
+    yz = o.swiglu_rows(rows, re, x, np.zeros_like(wgu), wd)
+    assert np.all(_bf16_val(yz) == 0)
+
+
+# ------------------------------------------------------------------ combine
+def pin_combine_identity_roundtrip(o):
+    """combine(dispatch(x)) with identity experts and renormalised weights is
+    x * sum(w) = x: within 1e-6 in fp32 and bit-exact after bf16 rounding."""
+    r = _rng(9)
+    n, e, k, ranks, d = 70, 16, 4, 4, 32
+    logits = r.standard_normal((n, e)).astype(np.float32)
+    idx, w = o.route(logits, k)
+    c = o.counts(idx, e)
+    off = o.offsets(n, e, k, ranks, c)
+    slot_of, _ = o.slots(idx, off, e)
+    x = r.standard_normal((n, d)).astype(np.float32)
+    recv = o.scatter_rows(x, slot_of, int(off[e]))
+    out = o.combine(recv, "f32", w, slot_of, "f32")
+    assert np.allclose(out, x, rtol=1e-6, atol=0)
+    xb = _bf16_bits(x)
+    recvb = o.scatter_rows(xb, slot_of, int(off[e]))
+    outb = o.combine(recvb, "bf16", w, slot_of, "bf16")
+    assert np.array_equal(outb, xb)
+
+
+def pin_combine_einsum(o):
+    """Weighted sum equals numpy's einsum over the gathered rows (float64,
+    then one rounding to fp32), element for element."""
+    r = _rng(10)
+    n, k, d, total = 25, 3, 40, 90
+    y = r.standard_normal((total, d)).astype(np.float32)
+    slot_of = np.stack([r.choice(total, k, replace=False) for _ in range(n)]).astype(np.int32)
+    w = r.uniform(0, 1, (n, k)).astype(np.float32)
+    out = o.combine(y, "f32", w, slot_of, "f32")
+    ref = np.einsum("tj,tjd->td", w.astype(np.float64), y.astype(np.float64)[slot_of])
+    assert np.array_equal(out, ref.astype(np.float32))
+    ab = o.combine_abs(y, "f32", w, slot_of)
+    assert np.allclose(ab, np.einsum("tj,tjd->td", w.astype(np.float64),
+                                     np.abs(y.astype(np.float64))[slot_of]), rtol=1e-15)
+
+
+def pin_hand_example(o):
+    """The hand-worked example in tests/golden/hand_example.json."""
+    with open(GOLDEN) as f:
+        g = json.load(f)
+    logits = np.array(g["logits"], np.float32)
+    k, e = g["top_k"], g["n_experts"]
+    idx, w = o.route(logits, k)
+    assert idx.tolist() == g["topk_idx"]
+    assert np.allclose(w, np.array(g["topk_w"]), rtol=0, atol=1e-7)
+    c = o.counts(idx, e)
+    assert c.tolist() == g["counts"]
+    x = np.array(g["x"], np.float32)
+    for lay in g["layouts"]:
+        off = o.offsets(g["n"], e, k, lay["n_ranks"], c)
+        assert off.tolist() == lay["expert_off"]
+        assert o.region_rows(g["n"], e, k, lay["n_ranks"]) == lay["region_rows"]
+        slot_of, src_of = o.slots(idx, off, e)
+        assert slot_of.tolist() == lay["slot_of"]
+        assert src_of.tolist() == lay["src_of"]
+        total = int(off[e])
+        ys = np.stack([np.arange(total), -np.arange(total)], 1).astype(np.float32)
+        out = o.combine(ys, "f32", w, slot_of, "f32")
+        assert np.allclose(out, np.array(lay["combine_with_y_slot"]), rtol=1e-6, atol=1e-6)
+        recv = o.scatter_rows(x, slot_of, total)
+        assert np.allclose(o.combine(recv, "f32", w, slot_of, "f32"), x, rtol=1e-6)
+
+
+def pin_run_path_tiny(o):
+    """The composed path on the tiny workload keeps every invariant: counts sum
+    to N*k, the slot map is a bijection, recv holds k copies of each row, and
+    combine(dispatch(x)) returns x."""
+    import workloads
+    cfg = workloads.CONFIGS["tiny"]
+    inp = {kk: workloads.as_numpy_bits(v) for kk, v in workloads.make_inputs(cfg).items()}
+    res = o.run_path(cfg, inp)
+    assert res["counts"].sum() == cfg.n * cfg.top_k
+    flat = res["slot_of"].ravel()
+    assert len(np.unique(flat)) == flat.size
+    assert np.array_equal(res["recv"][flat], np.repeat(inp["x"], cfg.top_k, axis=0))
+    assert np.allclose(res["out"], inp["x"], rtol=1e-6, atol=0)
+
+
+ALL_PINS = [v for kname, v in sorted(globals().items()) if kname.startswith("pin_")]
