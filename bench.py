@@ -1,0 +1,437 @@
+#!/usr/bin/env python
+"""Throughput of MoE dispatch + combine on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill]
+    python bench.py --impl reference ...   # the CPU oracle, timed on host cores
+
+A step is one pass of the hot path over one batch of synthetic tokens that is
+already resident in HBM: route (top-k + counts + scan) -> dispatch -> combine,
+three kernel launches.  The expert output Y that combine reads is produced
+once before timing by the identity expert (FP8 rows dequantised to bf16);
+it is an input of the dispatch+combine metric, like x.  L2 is flushed by a
+256 MiB write before every step, outside the timed events.  Each step is
+timed with CUDA events on the launching stream; the total over K steps is
+reduced with MAX across ranks.  With N > 1 every rank runs an independent
+replica on its own GPU (the path has no cross-GPU step on one GPU's virtual
+ranks), so scaling is weak and value = all ranks' tokens / max time.
+
+`e2e` times the public call a user makes, moe_layer, with pinned host
+buffers: host->device copies of logits, x and scales, the layer (route,
+dispatch, identity expert, combine) and the device->host copy of out.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+import torch.distributed as dist  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "dispatch+combine tokens/s and achieved HBM GB/s (% of B200 peak) on 1 GPU"
+FLUSH_BYTES = 256 << 20
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ------------------------------------------------------------------ accounting
+def algorithmic_bytes(cfg, n: int) -> dict:
+    """Bytes each step must move (index maps included; capacity, padding and
+    weights excluded)."""
+    xb = workloads.DTYPE_BYTES[cfg.x_dtype]
+    yb = workloads.DTYPE_BYTES[cfg.y_dtype]
+    ob = workloads.DTYPE_BYTES[cfg.out_dtype]
+    k, d, e = cfg.top_k, cfg.hidden, cfg.n_experts
+    row = d * xb + cfg.scale_cols * 4
+    route = n * e * 4 + n * k * 8
+    dispatch = n * row + n * k * row + n * k * 8
+    combine = n * k * d * yb + n * k * 8 + n * d * ob
+    return {"route": route, "dispatch": dispatch, "combine": combine,
+            "step": route + dispatch + combine}
+
+
+def describe(cfg, n: int) -> str:
+    s = (f"{cfg.name}: N={n}, D={cfg.hidden}, E={cfg.n_experts}, k={cfg.top_k}, "
+         f"R={cfg.n_ranks}, x={cfg.x_dtype}")
+    if cfg.scale_block:
+        s += f" + fp32 scale per {cfg.scale_block} cols"
+    s += f", Y={cfg.y_dtype}, out={cfg.out_dtype}, logits={cfg.logits}"
+    return s
+
+
+def read_peaks() -> tuple[float, str]:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("combine.cu", "moe_internal.cuh"):
+        with open(os.path.join(ROOT, "combine_moe_route_11_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per combine launch from the committed ncu summary, if it was
+    taken on the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            rec = json.load(f).get(workload)
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("source_hash") != kernel_source_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples (SM clock, throttle reasons) while the GPU works."""
+
+    FIELDS = ["clocks.sm", "clocks.max.sm", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.proc = None
+        self.window = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(device_index), "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), line.strip()))
+
+    def wait_first(self, timeout=5.0):
+        t0 = time.time()
+        while self.proc and not self.samples and time.time() - t0 < timeout:
+            time.sleep(0.05)
+
+    def stop(self, t_start: float, t_end: float):
+        if not self.proc:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ts, line in self.samples:
+            if not (t_start <= ts <= t_end):
+                continue
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[2:]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ distributed
+def init_dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and not dist.is_initialized():
+        import datetime
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def reduce_max(value: float, device) -> float:
+    """Max over ranks (identity without a process group)."""
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device):
+    if dist.is_available() and dist.is_initialized():
+        if device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+def time_oracle(cfg, budget_s: float, max_tokens: int, seed: int = 0):
+    """Tokens/s of the CPU oracle (route, dispatch, identity expert, combine)
+    on a sample sized to take about budget_s seconds."""
+    import oracle
+    cal_n = min(64, max_tokens)
+    inp = {k: workloads.as_numpy_bits(v) for k, v in
+           workloads.make_inputs(cfg, seed=seed, n=cal_n).items()}
+    t0 = time.perf_counter()
+    oracle.run_path(cfg, inp)
+    per_tok = (time.perf_counter() - t0) / cal_n
+    n = int(max(1, min(max_tokens, budget_s / max(per_tok, 1e-9))))
+    inp = {k: workloads.as_numpy_bits(v) for k, v in
+           workloads.make_inputs(cfg, seed=seed, n=n).items()}
+    t0 = time.perf_counter()
+    oracle.run_path(cfg, inp)
+    dt = time.perf_counter() - t0
+    return n, dt
+
+
+def run_reference(args, cfg):
+    world, rank, _ = init_dist()
+    if rank != 0:
+        return
+    n_steps = args.steps + args.warmup
+    per_step_budget = max(0.02, 90.0 / max(1, n_steps))
+    import oracle
+    cal = {k: workloads.as_numpy_bits(v) for k, v in
+           workloads.make_inputs(cfg, seed=0, n=16).items()}
+    t0 = time.perf_counter()
+    oracle.run_path(cfg, cal)
+    per_tok = (time.perf_counter() - t0) / 16
+    n = int(max(1, min(cfg.n, per_step_budget / max(per_tok, 1e-9))))
+    inp = {k: workloads.as_numpy_bits(v) for k, v in
+           workloads.make_inputs(cfg, seed=0, n=n).items()}
+    for _ in range(args.warmup):
+        oracle.run_path(cfg, inp)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.run_path(cfg, inp)
+    dt = time.perf_counter() - t0
+    value = n * args.steps / dt
+    sample = (f"{n} of the {cfg.n} tokens per step, the oracle's whole path "
+              f"(route, counts, offsets, slots, dispatch, identity expert, combine)")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt / args.steps * 1e3 * cfg.n / n, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": describe(cfg, cfg.n)},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_ours(args, cfg):
+    world, rank, local = init_dist()
+    import combine_moe_route_11_b200 as mr
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    n = cfg.n
+    plan = mr.Plan.from_config(cfg, n_max=n)
+    inp = workloads.make_inputs(cfg, seed=rank, n=n)
+    logits = inp["logits"].to(dev)
+    x = inp["x"].to(dev)
+    xs = inp["x_scale"].to(dev) if inp["x_scale"] is not None else None
+    ws = plan.new_workspace(dev)
+    b = plan.new_buffers(n, dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def route():
+        mr.moe_route_topk(plan, logits, b["topk_idx"], b["topk_w"], b["counts"],
+                          b["expert_off"], ws, stream)
+
+    def dispatch():
+        mr.moe_dispatch(plan, x, xs, b["topk_idx"], b["recv"], b["recv_scale"], b["slot_of"],
+                        b["src_of"], ws, stream)
+
+    # expert output read by combine: identity expert, produced once
+    route()
+    dispatch()
+    if cfg.x_dtype == "fp8_e4m3":
+        mr.moe_expert_dequant(plan, n, b["recv"], b["recv_scale"], b["slot_of"], b["y"], ws,
+                              stream)
+        y = b["y"]
+    else:
+        y = b["recv"]
+
+    def combine():
+        mr.moe_combine(plan, y, b["topk_w"], b["slot_of"], b["out"], ws, stream)
+
+    torch.cuda.synchronize(dev)
+    if mr.moe_get_status(plan, ws, stream) != 0:
+        raise RuntimeError("device status set before timing")
+
+    def step(evs=None):
+        flush.fill_(1)
+        if evs:
+            evs[0].record(stream)
+        route()
+        if evs:
+            evs[1].record(stream)
+        dispatch()
+        if evs:
+            evs[2].record(stream)
+        combine()
+        if evs:
+            evs[3].record(stream)
+
+    sampler = ClockSampler(local)
+    sampler.wait_first()
+    for _ in range(args.warmup):
+        step()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    t_start = time.time()
+    for i in range(args.steps):
+        step(ev[i])
+    torch.cuda.synchronize(dev)
+    t_end = time.time()
+    barrier(dev)
+    clocks = sampler.stop(t_start, t_end)
+    if mr.moe_get_status(plan, ws, stream) != 0:
+        raise RuntimeError("device status set during timing")
+    per = {"route": 0.0, "dispatch": 0.0, "combine": 0.0}
+    total_ms = 0.0
+    for e in ev:
+        per["route"] += e[0].elapsed_time(e[1])
+        per["dispatch"] += e[1].elapsed_time(e[2])
+        per["combine"] += e[2].elapsed_time(e[3])
+        total_ms += e[0].elapsed_time(e[3])
+    total_ms = reduce_max(total_ms, dev)
+    ms_step = total_ms / args.steps
+    nb = algorithmic_bytes(cfg, n)
+    peak, peak_kind = read_peaks()
+    kern_ms = {k: v / args.steps for k, v in per.items()}
+    dom = max(("dispatch", "combine"), key=lambda k: kern_ms[k])
+    achieved = nb[dom] / (kern_ms[dom] * 1e-3) / 1e9
+    step_gbs = nb["step"] / (ms_step * 1e-3) / 1e9
+
+    # ---- end to end through moe_layer with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        lws = plan.new_workspace(dev, layer=True)
+        logits_h = inp["logits"].pin_memory()
+        x_h = inp["x"].pin_memory()
+        xs_h = inp["x_scale"].pin_memory() if inp["x_scale"] is not None else None
+        out_d = torch.empty_like(b["out"])
+        out_h = torch.empty(out_d.shape, dtype=out_d.dtype).pin_memory()
+        logits_d, x_d = torch.empty_like(logits), torch.empty_like(x)
+        xs_d = torch.empty_like(xs) if xs is not None else None
+
+        def e2e_step():
+            logits_d.copy_(logits_h, non_blocking=True)
+            x_d.copy_(x_h, non_blocking=True)
+            if xs_d is not None:
+                xs_d.copy_(xs_h, non_blocking=True)
+            mr.moe_layer(plan, logits_d, x_d, xs_d, None, None, out_d, lws, stream)
+            out_h.copy_(out_d, non_blocking=True)
+
+        e2e_steps = max(3, min(args.steps, 50))
+        for _ in range(3):
+            e2e_step()
+        barrier(dev)
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        if mr.moe_get_status(plan, lws, stream) != 0:
+            raise RuntimeError("device status set during e2e")
+        e2e_ms = reduce_max(e0.elapsed_time(e1) / e2e_steps, dev)
+        h2d = logits_h.numel() * 4 + x_h.numel() * x_h.element_size() + \
+            (xs_h.numel() * 4 if xs_h is not None else 0)
+        d2h = out_h.numel() * out_h.element_size()
+        e2e = {"value": world * n / (e2e_ms * 1e-3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+               "steps": e2e_steps, "call": "moe_layer (identity experts)"}
+        del lws
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        nt, dt = time_oracle(cfg, budget_s=12.0, max_tokens=n)
+        cpu = {"value": nt / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+               "sample": f"{nt} of the {n} tokens of this workload, one pass of the oracle's "
+                         f"whole path (route, counts, offsets, slots, dispatch, identity expert, "
+                         f"combine) in {dt:.1f} s, single-threaded C"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": world * n / (ms_step * 1e-3), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic",
+            "config": {"workload": describe(cfg, n), "parallelism": f"replicas{world}",
+                       "l2": "flushed before every step by a 256 MiB write (untimed)",
+                       "timed": "route(top-k+counts+scan) + dispatch + combine, 3 launches/step",
+                       "y_source": "identity expert output, produced once before timing"},
+            "hbm_gbs": step_gbs, "hbm_pct_of_peak": 100.0 * step_gbs / peak,
+            "kernel_us": {k: v * 1e3 for k, v in kern_ms.items()},
+            "algorithmic_bytes": nb,
+            "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                         "traffic": recorded_traffic(cfg.name) if dom == "combine" else None},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": 3 * args.steps,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if dist.is_available() and dist.is_initialized():
+        dist.destroy_process_group()
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="prefill", choices=sorted(workloads.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    cfg = workloads.CONFIGS[args.workload]
+    if cfg.inter > 0:
+        ap.error("the dispatch+combine bench runs identity experts; choose another workload")
+    if args.impl == "reference":
+        run_reference(args, cfg)
+    else:
+        run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    main()

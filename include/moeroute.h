@@ -1,0 +1,212 @@
+/*
+ * moeroute -- Mixture-of-Experts token dispatch and combine on one B200.
+ *
+ * C ABI of libmoeroute.so.  Plain pointers and sizes only.
+ *
+ * The path (and the passages that define each step):
+ *   moe_route_topk   top-k experts per token, gate weights, per-expert counts
+ *                    and the rank-major expert offsets.  Rank-major buffers
+ *                    with fixed per-rank regions let every source compute its
+ *                    destinations locally, without exchanging metadata first
+ *                    ("One-Sided Expert-Parallel All-to-All for Mixture-of-
+ *                    Experts Inference over NVLink", abstract).  The selection
+ *                    has the [N, top_k] shape of the expert indices that the
+ *                    sorted/unsorted gather consumes ("backends/mlx: runtime
+ *                    MoE expert-sort for decode", Summary and author updates).
+ *   moe_dispatch     copies every token row to its k expert slots
+ *                    ("MLX expert parallelism all_to_all PR 3158", Facts:
+ *                    dispatch_local / dispatch_scatter_remote).
+ *   moe_expert_*     the expert step reading the dispatched buffer in place:
+ *                    grouped GEMMs read the rank-major buffer instead of a
+ *                    per-expert copy (arXiv 2611.13188 abstract); segments are
+ *                    contiguous, which is the promise a sorted-index grouped
+ *                    GEMM relies on ("backends/mlx: runtime MoE expert-sort
+ *                    for decode", author update on the gather_mm contract).
+ *   moe_combine      weighted sum of the k expert outputs back in token order
+ *                    (PR 3158 Facts: combine_gather_remote, combine_weighted_sum).
+ *   moe_layer        all of the above in order on one stream.
+ *
+ * Terms.  N = tokens of the call (n <= desc.n_max), D = hidden, E = experts,
+ * k = top_k, R = virtual ranks.  Virtual rank r owns experts
+ * [r*E/R, (r+1)*E/R) and the region of C_r = N*min(k, E/R) rows starting at
+ * row r*C_r of the receive buffer, which has T = R*C_r rows.  Inside a region
+ * experts ascend by id, inside an expert rows ascend by source token:
+ *     slot(t, j) = expert_off[e] + #{t' < t : t' picked e},  e = topk_idx[t, j].
+ * Rows of a region past its filled count are never written.
+ *
+ * Conventions for every entry point below.
+ *  - Memory: the caller allocates and owns every buffer; the library never
+ *    allocates or frees device memory.  "device" pointers must be device
+ *    memory of the current device, 16-byte aligned, rows dense (row stride =
+ *    D * element size).  Pointers named *_host are host memory.
+ *  - Asynchrony: compute calls only enqueue work on `stream` and return; none
+ *    synchronises except moe_get_status.  Results are visible after the usual
+ *    stream ordering.
+ *  - Errors: argument errors are detected on the host before anything is
+ *    enqueued and returned as MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED; a
+ *    failed launch returns MOE_ERR_CUDA.  Errors only the device can see (an
+ *    expert id outside [0, E) or a slot outside [0, T) in caller-supplied
+ *    arrays, a non-finite logit row) are recorded in the workspace status word
+ *    (first error wins), the offending item is skipped, and the outputs of
+ *    that call are unspecified.  moe_get_status returns and clears it.
+ *  - Workspace: `ws` is caller memory of moe_workspace_bytes() (or
+ *    moe_layer_workspace_bytes() for moe_layer), zero-filled before its first
+ *    use; the library keeps its control words consistent afterwards.  Calls
+ *    that share one workspace must be ordered on one stream.
+ */
+#ifndef MOEROUTE_H
+#define MOEROUTE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t (same underlying type); NULL is the legacy default stream. */
+typedef struct CUstream_st* moe_stream_t;
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = -1,   /* bad pointer, size, alignment or n > n_max */
+  MOE_ERR_UNSUPPORTED = -2,   /* valid but outside what this build implements */
+  MOE_ERR_CUDA = -3,          /* a CUDA runtime call or launch failed */
+  MOE_ERR_WORKSPACE = -4,     /* workspace too small or misaligned */
+  MOE_ERR_DEVICE_INDEX = -5,  /* device saw an expert id or slot out of range */
+  MOE_ERR_TIMEOUT = -6,       /* a bounded device-side wait gave up */
+  MOE_ERR_NONFINITE = -7      /* device saw a logit row with fewer than k finite values */
+} moe_status;
+
+typedef enum {
+  MOE_F32 = 0,       /* IEEE binary32 */
+  MOE_BF16 = 1,      /* bfloat16 */
+  MOE_FP8_E4M3 = 2   /* OCP FP8 E4M3 (finite, NaN = S.1111.111) */
+} moe_dtype;
+
+/* Static description of one MoE configuration. */
+typedef struct {
+  int32_t n_max;        /* largest N any call will pass (>= 1) */
+  int32_t hidden;       /* D */
+  int32_t n_experts;    /* E, 1..512 */
+  int32_t top_k;        /* k, 1..min(E, 32) */
+  int32_t n_ranks;      /* R >= 1, E % R == 0 */
+  int32_t x_dtype;      /* moe_dtype of token rows x (and of recv) */
+  int32_t y_dtype;      /* moe_dtype of expert outputs Y read by combine (F32|BF16) */
+  int32_t out_dtype;    /* moe_dtype of combine output (F32|BF16) */
+  int32_t scale_block;  /* FP8 rows: columns per fp32 scale (e.g. 128), 0 = no scales */
+  int32_t inter;        /* SwiGLU intermediate size I for moe_layer, 0 = identity experts */
+} moe_desc;
+
+typedef struct moe_plan moe_plan;
+
+/* Validate `desc` and build a plan (host only, no CUDA call).
+ * Requires: every row (x, Y, out) a multiple of 16 bytes; scale_block > 0
+ * only with FP8 rows and dividing D; T(n_max) < 2^31; for inter > 0 also
+ * x = y = BF16, D % 128 == 0 and I % 128 == 0.  *out is set only on MOE_OK. */
+MOE_API moe_status moe_plan_create(const moe_desc* desc, moe_plan** out);
+MOE_API void moe_plan_destroy(moe_plan* plan);
+
+/* Bytes of scratch for the route/dispatch/combine/expert calls (n <= n_max). */
+MOE_API size_t moe_workspace_bytes(const moe_plan* plan);
+/* Bytes of scratch for moe_layer: the above plus every intermediate buffer. */
+MOE_API size_t moe_layer_workspace_bytes(const moe_plan* plan);
+/* C_r and T for a call with n tokens (rows per region, rows of recv). */
+MOE_API int64_t moe_region_rows(const moe_plan* plan, int32_t n);
+MOE_API int64_t moe_recv_rows(const moe_plan* plan, int32_t n);
+
+/* Route: for each token t < n,
+ *   topk_idx[t, 0..k)  experts by descending logit, ties to the lower id;
+ *   topk_w[t, j]       = exp(L[t,idx_j] - L[t,idx_0]) / sum_i exp(L[t,idx_i] - L[t,idx_0]);
+ *   counts[e]          = #{(t, j) : topk_idx[t, j] == e};
+ *   expert_off[e]      = (e / (E/R)) * C_r + sum of counts of lower experts
+ *                        of the same rank;  expert_off[E] = T.
+ * logits: device fp32 [n, E] row-major.  topk_idx: device int32 [n, k];
+ * topk_w: device fp32 [n, k]; counts: device int32 [E]; expert_off: device
+ * int32 [E + 1].  Also leaves in `ws` the per-block bases that moe_dispatch
+ * uses for the slots of this routing.  n = 0 writes zero counts and offsets. */
+MOE_API moe_status moe_route_topk(const moe_plan* plan, int32_t n, const float* logits,
+                          int32_t* topk_idx, float* topk_w, int32_t* counts,
+                          int32_t* expert_off, void* ws, moe_stream_t stream);
+
+/* Dispatch: recv[slot(t, j)] = x[t] (D elements of x_dtype, copied as bytes),
+ * recv_scale[slot(t, j)] = x_scale[t] (D / scale_block fp32, when scale_block
+ * > 0), slot_of[t, j] = slot(t, j), src_of[slot(t, j)] = t*k + j.
+ * Must follow moe_route_topk on the same stream with the same n, topk_idx and
+ * ws (the slots come from that call's per-block bases).  x: device [n, D];
+ * x_scale: device fp32 [n, D/scale_block] or NULL when scale_block == 0;
+ * recv: device [T, D]; recv_scale: device fp32 [T, D/scale_block] or NULL;
+ * slot_of: device int32 [n, k]; src_of: device int32 [T] (only filled slots
+ * are written). */
+MOE_API moe_status moe_dispatch(const moe_plan* plan, int32_t n, const void* x, const float* x_scale,
+                        const int32_t* topk_idx, void* recv, float* recv_scale,
+                        int32_t* slot_of, int32_t* src_of, void* ws, moe_stream_t stream);
+
+/* Identity expert for FP8 rows: Y[s, c] = round_y(code[s, c] * recv_scale[s,
+ * c / scale_block]) for every filled slot s = slot_of[t, j], correctly rounded
+ * (to nearest even) from the exact product.  recv: device e4m3 [T, D];
+ * recv_scale: device fp32 [T, D/scale_block] (NULL = scale 1); y: device
+ * y_dtype [T, D]. */
+MOE_API moe_status moe_expert_dequant(const moe_plan* plan, int32_t n, const void* recv,
+                              const float* recv_scale, const int32_t* slot_of, void* y,
+                              void* ws, moe_stream_t stream);
+
+/* SwiGLU experts read in place from the rank-major buffer: for every expert e
+ * and row s in [expert_off[e], expert_off[e] + counts[e]):
+ *   h[s, :] = bf16( silu(recv[s] . Wg[e]^T) * (recv[s] . Wu[e]^T) ),
+ *   y[s, :] = bf16( h[s] . Wd[e]^T ),   silu(z) = z / (1 + exp(-z)),
+ * fp32 accumulation on the tensor cores.  w_gate_up: device bf16 [E, 2I, D]
+ * (rows [0, I) are Wg[e], rows [I, 2I) are Wu[e]); w_down: device bf16
+ * [E, D, I]; recv: device bf16 [T, D]; h: device bf16 [T, I]; y: device bf16
+ * [T, D].  counts and expert_off as written by moe_route_topk. */
+MOE_API moe_status moe_expert_swiglu(const moe_plan* plan, int32_t n, const void* recv,
+                             const int32_t* counts, const int32_t* expert_off,
+                             const void* w_gate_up, const void* w_down, void* h, void* y,
+                             void* ws, moe_stream_t stream);
+
+/* Combine: out[t, c] = sum_{j=0}^{k-1} topk_w[t, j] * Y[slot_of[t, j], c],
+ * accumulated in fp32 with fused multiply-adds in increasing j, then rounded
+ * to nearest even into out_dtype.  y: device y_dtype [T, D]; topk_w: device
+ * fp32 [n, k]; slot_of: device int32 [n, k]; out: device out_dtype [n, D]. */
+MOE_API moe_status moe_combine(const moe_plan* plan, int32_t n, const void* y, const float* topk_w,
+                       const int32_t* slot_of, void* out, void* ws, moe_stream_t stream);
+
+/* The whole layer on one stream: route -> dispatch -> expert -> combine.
+ * Experts are SwiGLU when desc.inter > 0 (w_gate_up, w_down as in
+ * moe_expert_swiglu), else identity (FP8 rows dequantised, other rows read
+ * as Y directly; then y_dtype must equal x_dtype).  logits: device fp32
+ * [n, E]; x, x_scale as in moe_dispatch; out: device out_dtype [n, D];
+ * ws: moe_layer_workspace_bytes() of zero-filled device memory, which holds
+ * every intermediate (see moe_layer_buffer). */
+MOE_API moe_status moe_layer(const moe_plan* plan, int32_t n, const float* logits, const void* x,
+                     const float* x_scale, const void* w_gate_up, const void* w_down,
+                     void* out, void* ws, moe_stream_t stream);
+
+/* Where moe_layer keeps an intermediate inside its workspace, so a caller
+ * can read it after the call: returns ws + byte offset, or NULL for an
+ * unknown name.  Names: "topk_idx", "topk_w", "counts", "expert_off",
+ * "slot_of", "src_of", "recv", "recv_scale", "y", "h". */
+MOE_API void* moe_layer_buffer(const moe_plan* plan, void* ws, const char* name);
+
+/* Read and clear the device status word of `ws`: synchronises `stream`,
+ * returns MOE_OK or the first device-detected error since the last call
+ * (MOE_ERR_CUDA if the copy itself fails). */
+MOE_API moe_status moe_get_status(const moe_plan* plan, void* ws, moe_stream_t stream);
+
+/* Zero the control words of a workspace (an alternative to zero-filling
+ * it), enqueued on `stream`. */
+MOE_API moe_status moe_workspace_init(const moe_plan* plan, void* ws, moe_stream_t stream);
+
+/* Human-readable name of a status code (static string). */
+MOE_API const char* moe_strerror(moe_status status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOEROUTE_H */

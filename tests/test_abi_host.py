@@ -1,0 +1,119 @@
+"""The C-ABI library without a GPU: it loads, exports every symbol that
+include/moeroute.h declares, and its host-side validation behaves as the
+header states.  No call here reaches a CUDA launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moeroute.h")
+
+
+def build_library():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_moeroute_build", os.path.join(ROOT, "combine_moe_route_11_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod.build()
+
+
+@pytest.fixture(scope="module")
+def mr():
+    build_library()
+    import combine_moe_route_11_b200 as m
+    return m
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_header_declares_the_path():
+    names = declared_functions()
+    for must in ["moe_route_topk", "moe_dispatch", "moe_combine", "moe_layer",
+                 "moe_expert_swiglu", "moe_expert_dequant", "moe_plan_create",
+                 "moe_get_status", "moe_strerror"]:
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(mr):
+    lib = ctypes.CDLL(mr.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def _plan_code(mr, **kw):
+    base = dict(n_max=64, hidden=256, n_experts=8, top_k=2, n_ranks=2, x_dtype=0, y_dtype=0,
+                out_dtype=0, scale_block=0, inter=0)
+    base.update(kw)
+    d = mr._Desc(*[base[f] for f, _ in mr._Desc._fields_])
+    h = ctypes.c_void_p()
+    rc = mr._lib.moe_plan_create(ctypes.byref(d), ctypes.byref(h))
+    if rc == 0:
+        mr._lib.moe_plan_destroy(h)
+    return rc
+
+
+@pytest.mark.parametrize("kw,code", [
+    ({}, 0),
+    ({"n_max": 0}, -1),
+    ({"top_k": 9}, -1),                       # k > E
+    ({"n_ranks": 3}, -1),                     # E % R != 0
+    ({"hidden": 250}, -1),                    # fp32 row of 1000 bytes, not 16-byte whole
+    ({"x_dtype": 1, "y_dtype": 1, "out_dtype": 1, "hidden": 8}, 0),
+    ({"x_dtype": 2, "hidden": 16, "scale_block": 16, "y_dtype": 1, "out_dtype": 1}, 0),
+    ({"x_dtype": 2, "hidden": 256, "scale_block": 12, "y_dtype": 1, "out_dtype": 1}, -1),
+    ({"scale_block": 128}, -1),               # scales only with FP8 rows
+    ({"n_experts": 1024, "top_k": 2, "n_ranks": 1}, -2),
+    ({"top_k": 33, "n_experts": 64}, -2),
+    ({"y_dtype": 2}, -2),
+    ({"inter": 128}, -2),                     # SwiGLU needs bf16 rows
+    ({"inter": 128, "x_dtype": 1, "y_dtype": 1, "out_dtype": 1}, 0),
+    ({"inter": 100, "x_dtype": 1, "y_dtype": 1, "out_dtype": 1}, -2),
+    ({"n_max": 1 << 27, "n_experts": 256, "top_k": 8, "n_ranks": 8}, -2),  # T >= 2^31
+])
+def test_plan_validation(mr, kw, code):
+    assert _plan_code(mr, **kw) == code
+
+
+def test_capacity_and_workspace(mr):
+    import oracle
+    for (n_max, e, k, r) in [(64, 8, 2, 2), (4096, 256, 8, 8), (100, 8, 4, 4), (77, 12, 3, 3)]:
+        p = mr.Plan(n_max, 256, e, k, r, "f32", "f32", "f32")
+        for n in (0, 1, n_max // 2, n_max):
+            assert p.region_rows(n) == oracle.region_rows(n, e, k, r)
+            assert p.recv_rows(n) == r * oracle.region_rows(n, e, k, r)
+        assert p.region_rows(n_max + 1) == -1
+        assert p.workspace_bytes > 0 and p.workspace_bytes % 256 == 0
+        assert p.layer_workspace_bytes > p.workspace_bytes
+        p.close()
+
+
+def test_host_argument_errors_return_before_any_launch(mr):
+    p = mr.Plan(64, 256, 8, 2, 2, "f32", "f32", "f32")
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: every call below fails validation
+    lib = mr._lib
+    assert lib.moe_route_topk(p.handle, 65, fake, fake, fake, fake, fake, fake, None) == -1
+    assert lib.moe_route_topk(p.handle, -1, fake, fake, fake, fake, fake, fake, None) == -1
+    assert lib.moe_route_topk(p.handle, 4, fake, fake, fake, fake, fake,
+                              ctypes.c_void_p((1 << 20) + 16), None) == -4  # ws misaligned
+    assert lib.moe_route_topk(p.handle, 4, fake, fake, fake, None, fake, fake, None) == -1
+    assert lib.moe_dispatch(p.handle, 4, ctypes.c_void_p((1 << 20) + 8), None, fake, fake, None,
+                            fake, fake, fake, None) == -1          # x not 16-byte aligned
+    assert lib.moe_dispatch(p.handle, 0, None, None, None, None, None, None, None, fake,
+                            None) == 0                               # n = 0 is a no-op
+    assert lib.moe_combine(p.handle, 65, fake, fake, fake, fake, fake, None) == -1
+    assert lib.moe_expert_dequant(p.handle, 4, fake, fake, fake, fake, fake, None) == -2
+    assert lib.moe_expert_swiglu(p.handle, 4, fake, fake, fake, fake, fake, fake, fake, fake,
+                                 None) == -2
+    assert lib.moe_layer_buffer(p.handle, fake, b"nope") is None
+    assert lib.moe_layer_buffer(p.handle, fake, b"recv") is not None
+    assert lib.moe_get_status(None, fake, None) == -1
+    for code in range(-7, 1):
+        assert mr.moe_strerror(code) not in ("", "unknown status")
+    p.close()
