@@ -8,10 +8,13 @@ A step is one pass of the hot path over one batch of synthetic tokens that is
 already resident in HBM: route (top-k + counts + scan) -> dispatch -> combine,
 three kernel launches.  The expert output Y that combine reads is produced
 once before timing by the identity expert (FP8 rows dequantised to bf16);
-it is an input of the dispatch+combine metric, like x.  L2 is flushed by a
-256 MiB write before every step, outside the timed events.  Each step is
-timed with CUDA events on the launching stream; the total over K steps is
-reduced with MAX across ranks.  With N > 1 every rank runs an independent
+it is an input of the dispatch+combine metric, like x.  No step finds its
+inputs in L2: a step moves more than 4x the L2 size, or else enough buffer
+sets rotate that 4x L2 of traffic separates two uses of a set.  Steps run
+back to back; the K-step region is timed with CUDA events on the launching
+stream and reduced with MAX across ranks.  Kernel durations (for the
+roofline) come from a separate pass with events between the kernels, which
+would otherwise break the programmatic-launch overlap between them.  With N > 1 every rank runs an independent
 replica on its own GPU (the path has no cross-GPU step on one GPU's virtual
 ranks), so scaling is weak and value = all ranks' tokens / max time.
 
@@ -40,7 +43,7 @@ import torch.distributed as dist  # noqa: E402
 import workloads  # noqa: E402
 
 METRIC = "dispatch+combine tokens/s and achieved HBM GB/s (% of B200 peak) on 1 GPU"
-FLUSH_BYTES = 256 << 20
+L2_BYTES = 126 << 20
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -257,84 +260,104 @@ def run_ours(args, cfg):
     stream = torch.cuda.current_stream(dev)
     n = cfg.n
     plan = mr.Plan.from_config(cfg, n_max=n)
-    inp = workloads.make_inputs(cfg, seed=rank, n=n)
-    logits = inp["logits"].to(dev)
-    x = inp["x"].to(dev)
-    xs = inp["x_scale"].to(dev) if inp["x_scale"] is not None else None
-    ws = plan.new_workspace(dev)
-    b = plan.new_buffers(n, dev)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    nb = algorithmic_bytes(cfg, n)
+    # Buffer sets rotate so that a step never finds its data in L2: the other
+    # sets' traffic between two uses of a set is at least 4x the L2 size.
+    n_sets = max(1, min(32, -(-4 * L2_BYTES // nb["step"]) + 1)) if nb["step"] < 4 * L2_BYTES else 1
+    sets = []
+    for si in range(n_sets):
+        inp = workloads.make_inputs(cfg, seed=rank * 1000 + si, n=n)
+        st = {"inp": inp, "logits": inp["logits"].to(dev), "x": inp["x"].to(dev),
+              "xs": inp["x_scale"].to(dev) if inp["x_scale"] is not None else None,
+              "ws": plan.new_workspace(dev), "b": plan.new_buffers(n, dev)}
+        sets.append(st)
 
-    def route():
-        mr.moe_route_topk(plan, logits, b["topk_idx"], b["topk_w"], b["counts"],
-                          b["expert_off"], ws, stream)
+    def route(st):
+        b = st["b"]
+        mr.moe_route_topk(plan, st["logits"], b["topk_idx"], b["topk_w"], b["counts"],
+                          b["expert_off"], st["ws"], stream)
 
-    def dispatch():
-        mr.moe_dispatch(plan, x, xs, b["topk_idx"], b["recv"], b["recv_scale"], b["slot_of"],
-                        b["src_of"], ws, stream)
+    def dispatch(st):
+        b = st["b"]
+        mr.moe_dispatch(plan, st["x"], st["xs"], b["topk_idx"], b["recv"], b["recv_scale"],
+                        b["slot_of"], b["src_of"], st["ws"], stream)
 
-    # expert output read by combine: identity expert, produced once
-    route()
-    dispatch()
-    if cfg.x_dtype == "fp8_e4m3":
-        mr.moe_expert_dequant(plan, n, b["recv"], b["recv_scale"], b["slot_of"], b["y"], ws,
-                              stream)
-        y = b["y"]
-    else:
-        y = b["recv"]
+    def combine(st):
+        b = st["b"]
+        mr.moe_combine(plan, st["y"], b["topk_w"], b["slot_of"], b["out"], st["ws"], stream)
 
-    def combine():
-        mr.moe_combine(plan, y, b["topk_w"], b["slot_of"], b["out"], ws, stream)
-
+    # expert output read by combine: identity expert, produced once per set
+    for st in sets:
+        route(st)
+        dispatch(st)
+        b = st["b"]
+        if cfg.x_dtype == "fp8_e4m3":
+            mr.moe_expert_dequant(plan, n, b["recv"], b["recv_scale"], b["slot_of"], b["y"],
+                                  st["ws"], stream)
+            st["y"] = b["y"]
+        else:
+            st["y"] = b["recv"]
     torch.cuda.synchronize(dev)
-    if mr.moe_get_status(plan, ws, stream) != 0:
-        raise RuntimeError("device status set before timing")
+    for st in sets:
+        if mr.moe_get_status(plan, st["ws"], stream) != 0:
+            raise RuntimeError("device status set before timing")
 
-    def step(evs=None):
-        flush.fill_(1)
+    def step(st, evs=None):
         if evs:
             evs[0].record(stream)
-        route()
+        route(st)
         if evs:
             evs[1].record(stream)
-        dispatch()
+        dispatch(st)
         if evs:
             evs[2].record(stream)
-        combine()
+        combine(st)
         if evs:
             evs[3].record(stream)
 
-    sampler = ClockSampler(local)
-    sampler.wait_first()
-    for _ in range(args.warmup):
-        step()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    barrier(dev)
+    for i in range(args.warmup):
+        step(sets[i % n_sets])
+    # pass 1: per-kernel CUDA events inside every step (kernel durations)
+    k_steps = min(args.steps, 200)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(k_steps)]
     torch.cuda.synchronize(dev)
-    t_start = time.time()
-    for i in range(args.steps):
-        step(ev[i])
+    for i in range(k_steps):
+        step(sets[i % n_sets], ev[i])
     torch.cuda.synchronize(dev)
-    t_end = time.time()
-    barrier(dev)
-    clocks = sampler.stop(t_start, t_end)
-    if mr.moe_get_status(plan, ws, stream) != 0:
-        raise RuntimeError("device status set during timing")
     per = {"route": 0.0, "dispatch": 0.0, "combine": 0.0}
-    total_ms = 0.0
     for e in ev:
         per["route"] += e[0].elapsed_time(e[1])
         per["dispatch"] += e[1].elapsed_time(e[2])
         per["combine"] += e[2].elapsed_time(e[3])
-        total_ms += e[0].elapsed_time(e[3])
-    total_ms = reduce_max(total_ms, dev)
+    kern_ms = {k: v / k_steps for k, v in per.items()}
+    # pass 2: K steps back to back, events only around the region
+    sampler = ClockSampler(local)
+    sampler.wait_first()
+    for i in range(args.warmup):
+        step(sets[i % n_sets])
+    r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    t_start = time.time()
+    r0.record(stream)
+    for i in range(args.steps):
+        step(sets[i % n_sets])
+    r1.record(stream)
+    torch.cuda.synchronize(dev)
+    t_end = time.time()
+    barrier(dev)
+    clocks = sampler.stop(t_start, t_end)
+    for st in sets:
+        if mr.moe_get_status(plan, st["ws"], stream) != 0:
+            raise RuntimeError("device status set during timing")
+    total_ms = reduce_max(r0.elapsed_time(r1), dev)
     ms_step = total_ms / args.steps
-    nb = algorithmic_bytes(cfg, n)
     peak, peak_kind = read_peaks()
-    kern_ms = {k: v / args.steps for k, v in per.items()}
     dom = max(("dispatch", "combine"), key=lambda k: kern_ms[k])
     achieved = nb[dom] / (kern_ms[dom] * 1e-3) / 1e9
     step_gbs = nb["step"] / (ms_step * 1e-3) / 1e9
+    inp = sets[0]["inp"]
+    logits, x, xs, b = sets[0]["logits"], sets[0]["x"], sets[0]["xs"], sets[0]["b"]
 
     # ---- end to end through moe_layer with pinned host buffers
     e2e = None
@@ -393,7 +416,9 @@ def run_ours(args, cfg):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic",
             "config": {"workload": describe(cfg, n), "parallelism": f"replicas{world}",
-                       "l2": "flushed before every step by a 256 MiB write (untimed)",
+                       "l2": (f"no flush: {n_sets} buffer set(s) rotate so a step's data "
+                              f"was last touched >= 4x L2 ({nb['step'] * max(1, n_sets - 1) / 1e6:.0f}"
+                              f" MB of traffic) earlier; steps run back to back"),
                        "timed": "route(top-k+counts+scan) + dispatch + combine, 3 launches/step",
                        "y_source": "identity expert output, produced once before timing"},
             "hbm_gbs": step_gbs, "hbm_pct_of_peak": 100.0 * step_gbs / peak,
@@ -421,10 +446,14 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override N (smaller batches for profiler captures only)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     cfg = workloads.CONFIGS[args.workload]
+    if args.tokens:
+        cfg = cfg.replace(n=args.tokens)
     if cfg.inter > 0:
         ap.error("the dispatch+combine bench runs identity experts; choose another workload")
     if args.impl == "reference":

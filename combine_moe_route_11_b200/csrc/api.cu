@@ -21,6 +21,25 @@ int num_sms() {
   return v;
 }
 
+cudaError_t set_smem_limit(const void* kernel, int bytes) {
+  // (kernel, device) pairs already raised; a handful of kernels, few devices
+  static const void* done_k[64];
+  static int done_d[64];
+  static int done_n = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  for (int i = 0; i < done_n; ++i)
+    if (done_k[i] == kernel && done_d[i] == dev) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && done_n < 64) {
+    done_k[done_n] = kernel;
+    done_d[done_n] = dev;
+    ++done_n;
+  }
+  return e;
+}
+
 namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -36,6 +55,7 @@ Layout make_layout(const moe_plan& p) {
   };
   L.ctrl = take(sizeof(Ctrl));
   L.blk = take(size_t(p.blocks_max) * d.n_experts * 4);
+  L.bases = take(size_t(p.blocks_max) * d.n_experts * 4);
   L.rank = take(size_t(d.n_max) * d.top_k);
   L.route_end = at;
   const size_t nk = size_t(d.n_max) * d.top_k;
@@ -136,6 +156,7 @@ moe_status moe_route_topk(const moe_plan* p, int32_t n, const float* logits, int
   if (s != MOE_OK) return s;
   if (!counts || !expert_off || (n > 0 && (!logits || !topk_idx || !topk_w)))
     return MOE_ERR_INVALID_ARG;
+  if (n > 0 && !aligned16(logits)) return MOE_ERR_INVALID_ARG;
   return cuda_status(launch_route(*p, n, logits, topk_idx, topk_w, counts, expert_off, ws,
                                   reinterpret_cast<cudaStream_t>(stream)));
 }

@@ -11,20 +11,24 @@
 
 namespace moe {
 
-// Tokens per route block.  One block's tokens form two 32-token groups whose
-// membership masks give each (token, expert) pair its rank inside the block.
-constexpr int kRouteTokens = 64;
-constexpr int kRouteThreads = 256;
+// Tokens per route block: one warp per token, and the block's 32 tokens form
+// the membership masks that give each (token, expert) pair its in-block rank.
+constexpr int kRouteTokens = 32;
+constexpr int kRouteThreads = 1024;
 constexpr int kMaxExperts = 512;
 constexpr int kMaxTopK = 32;
 
 // Control words at the start of every workspace.
 struct Ctrl {
-  unsigned int ticket;  // route blocks finished so far (reset by the last one)
+  unsigned int arrive;  // grid barrier: blocks arrived (reset by the last one)
   int status;           // first device-detected error, 0 = none
-  unsigned int pad[62];
+  unsigned int gen;     // grid barrier: generation, bumped when all arrived
+  unsigned int pad[61];
 };
 static_assert(sizeof(Ctrl) == 256, "control block is 256 bytes");
+
+__host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+__host__ __device__ __forceinline__ int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -34,7 +38,7 @@ inline int elem_bytes(int dtype) {
 
 // Byte offsets of every buffer inside a workspace, fixed by n_max.
 struct Layout {
-  size_t ctrl, blk, rank, route_end;
+  size_t ctrl, blk, bases, rank, route_end;
   size_t topk_idx, topk_w, counts, expert_off, slot_of, src_of, recv, recv_scale, y, h, end;
 };
 
@@ -58,6 +62,8 @@ inline int64_t total_rows(const moe_plan& p, int32_t n) { return region_rows(p, 
 inline int route_blocks(int32_t n) { return n <= 0 ? 1 : (n + kRouteTokens - 1) / kRouteTokens; }
 
 int num_sms();  // of the current device (cached per device)
+// Raise a kernel's dynamic shared-memory limit once per device.
+cudaError_t set_smem_limit(const void* kernel, int bytes);
 
 // Launchers (return cudaGetLastError()).
 cudaError_t launch_route(const moe_plan& p, int32_t n, const float* logits, int32_t* topk_idx,
@@ -74,12 +80,78 @@ cudaError_t launch_swiglu(const moe_plan& p, int32_t n, const void* recv, const 
                           const int32_t* expert_off, const void* w_gate_up, const void* w_down,
                           void* h, void* y, void* ws, cudaStream_t st);
 
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while the previous kernel of the stream finishes, and must call
+// grid_dependency_wait() before its first global-memory access.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // ------------------------------------------------------------------ device helpers
 #ifdef __CUDACC__
+
+// Wait until the grids this one depends on have completed and their memory
+// is visible (a no-op without a programmatic dependency).
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Allow the next kernel of the stream to be scheduled (it still waits for
+// this grid's completion before touching memory).
+__device__ __forceinline__ void grid_dependents_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 
 __device__ __forceinline__ void set_status(void* ws, int code) {
   Ctrl* c = reinterpret_cast<Ctrl*>(ws);
   atomicCAS(&c->status, 0, code);
+}
+
+// Barrier across all `blocks` blocks of a grid whose blocks are all resident
+// (cooperative launch).  The wait is bounded (~2^31 cycles); on timeout it
+// records MOE_ERR_TIMEOUT and returns false, and the workspace must be
+// re-initialised before its next use.
+__device__ __forceinline__ bool grid_barrier(void* ws, unsigned blocks) {
+  __shared__ int s_ok;
+  Ctrl* c = reinterpret_cast<Ctrl*>(ws);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    bool ok = true;
+    __threadfence();
+    const unsigned gen = *reinterpret_cast<volatile unsigned*>(&c->gen);
+    __threadfence();
+    if (atomicAdd(&c->arrive, 1u) + 1u == blocks) {
+      atomicExch(&c->arrive, 0u);
+      __threadfence();
+      atomicAdd(&c->gen, 1u);
+    } else {
+      const long long t0 = clock64();
+      while (*reinterpret_cast<volatile unsigned*>(&c->gen) == gen) {
+        if (clock64() - t0 > (1ll << 31)) {
+          ok = false;
+          set_status(ws, MOE_ERR_TIMEOUT);
+          break;
+        }
+        __nanosleep(32);
+      }
+    }
+    __threadfence();
+    s_ok = ok;
+  }
+  __syncthreads();
+  return s_ok != 0;
 }
 
 // 16-byte global load through the non-coherent path, not kept in L1.
@@ -96,6 +168,88 @@ __device__ __forceinline__ void st_cs_v4(void* p, const uint4& v) {
   asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y),
                "r"(v.z), "r"(v.w)
                : "memory");
+}
+
+// ---- bulk asynchronous copies (TMA engine) and mbarriers, no multicast
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+               : "memory");
+}
+
+// Make mbarrier initialisation visible to the async proxy.
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+// Order this thread's generic-proxy shared-memory accesses before later
+// async-proxy (bulk copy) accesses of the same bytes, and vice versa.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for an mbarrier phase: gives up after ~2^31 SM cycles
+// (about a second) and returns false.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity))
+    if (clock64() - t0 > (1ll << 31)) return false;
+  return true;
+}
+
+// global -> shared bulk copy completing on an mbarrier (bytes % 16 == 0,
+// both addresses 16-byte aligned).
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_addr(smem_dst)),
+      "l"(gsrc), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// shared -> global bulk copy tracked by this thread's bulk groups.
+__device__ __forceinline__ void bulk_store(void* gdst, const void* smem_src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
+               "r"(smem_addr(smem_src)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Wait until at most N of this thread's bulk groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+// Wait until all of this thread's bulk groups have completed.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }

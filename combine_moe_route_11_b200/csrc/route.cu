@@ -10,28 +10,34 @@
 // ("backends/mlx: runtime MoE expert-sort for decode", author update on the
 // sorted branch) -- computed here as a counting sort, without any sort.
 //
-// One launch, three phases:
-//  1. each warp routes tokens: the k largest logits by k rounds of a warp
-//     argmax (lower expert id wins a tie), then a softmax over the k winners;
-//  2. each block (64 tokens = two 32-token groups) builds, per expert, a
-//     bitmask of the tokens of each group that picked it; the rank of token t
-//     among the block's tokens picking e is a popcount of the lower lanes, and
-//     the block's count of e is the popcount of the whole mask;
-//  3. the last block to finish (ticket counter) scans the [blocks, E] count
-//     table: expert totals, the rank-major expert offsets, and in place the
-//     base slot of every (block, expert).
-// All integer results are deterministic: no atomics decide an order.
+// One cooperative launch (all blocks resident), two phases split by a
+// bounded grid barrier:
+//  1. per route block of 32 tokens, one warp per token: the k largest logits
+//     by k rounds of a warp argmax on order-preserving integer keys (two
+//     single-instruction warp reductions per round; the lower expert id wins
+//     a tie) and a softmax over the k winners; then, per expert, the bitmask
+//     of the block's tokens that picked it gives each (token, expert) pair
+//     its rank among the block's tokens (popcount of the lower lanes) and the
+//     block's count of the expert;
+//  2. per column of (up to) 4 experts: the count columns of the experts of
+//     its rank below its own give the rank-major offsets, and an exclusive
+//     scan of its own columns over the route blocks gives each block's
+//     absolute base slot (a separate table: other blocks still read counts).
+// A slot is then base[block][e] + rank.  All integer results are
+// deterministic: no atomic decides an order.
 #include "moe_internal.cuh"
 
 #include <float.h>
 #include <limits.h>
+
+#include <type_traits>
 
 namespace moe {
 namespace {
 
 constexpr unsigned kFull = 0xFFFFFFFFu;
 constexpr int kWarps = kRouteThreads / 32;
-constexpr int kTokPerWarp = kRouteTokens / kWarps;
+constexpr int kMaxSpan = kMaxExperts + 4;
 
 struct RouteArgs {
   const float* logits;
@@ -39,213 +45,283 @@ struct RouteArgs {
   float* topk_w;
   int32_t* counts;
   int32_t* expert_off;
-  int32_t* blk;    // [blocks, E]: block counts, rewritten as block bases
+  int32_t* blk;    // [blocks, E] per-block counts
+  int32_t* bases;  // [blocks, E] per-block absolute base slots
   uint8_t* rank;   // [n, k]: rank of (t, j) among the block's tokens picking e
   void* ws;
   int32_t n, E, K, R;
+  int32_t blocks;       // route blocks B = ceil(n / 32), at least 1
   int32_t region_rows;  // C_r
 };
 
-template <int VPL>
-__device__ __forceinline__ void route_token(const RouteArgs& a, const float (&v)[VPL], int t,
-                                            int tl, int lane, int32_t* s_sel) {
+// Order-preserving unsigned key of a finite float (larger float -> larger
+// key; -0 and +0 share a key so they tie; finite keys are >= 0x00800000).
+// Non-finite logits get key 1, below every finite one, so they are picked
+// only when fewer than k finite logits remain (lowest id first) and flag the
+// row.  Key 0 marks padding and experts already picked.
+__device__ __forceinline__ uint32_t order_key(float f) {
+  if (!isfinite(f)) return 1u;
+  uint32_t b = __float_as_uint(f);
+  if (b == 0x80000000u) b = 0u;
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+__device__ __forceinline__ float key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+// Expert held in value slot q of `lane`.  VEC = 4: lane l holds experts
+// 128*(q/4) + 4l + q%4 (loaded as float4; E % 128 == 0).  VEC = 1: expert
+// 32q + l.  Either way the expert id grows with q for a fixed lane.
+template <int VEC>
+__device__ __forceinline__ int expert_of(int q, int lane) {
+  if constexpr (VEC == 4) return (q >> 2) * 128 + lane * 4 + (q & 3);
+  else return q * 32 + lane;
+}
+
+// Top-k and softmax of token t by the calling warp; returns lane j's pick.
+template <int VPL, int VEC>
+__device__ __forceinline__ int route_token(const RouteArgs& a, int64_t t, int lane) {
   const int E = a.E, K = a.K;
-  uint32_t picked = 0;
-  float my_v = -INFINITY;
-  int my_i = 0;
-  bool nonfinite = false;
-  for (int j = 0; j < K; ++j) {
-    // best remaining (value, id) of this lane; ids ascend with q, so a strict
-    // compare keeps the lowest id among equal values
-    float bv = -INFINITY;
-    int bi = INT_MAX;
+  const float* row = a.logits + t * E;
+  uint32_t key[VPL];
+  if constexpr (VEC == 4) {
+#pragma unroll
+    for (int q4 = 0; q4 < VPL / 4; ++q4) {
+      const float4 v = __ldcs(reinterpret_cast<const float4*>(row + q4 * 128) + lane);
+      key[4 * q4 + 0] = order_key(v.x);
+      key[4 * q4 + 1] = order_key(v.y);
+      key[4 * q4 + 2] = order_key(v.z);
+      key[4 * q4 + 3] = order_key(v.w);
+    }
+  } else {
 #pragma unroll
     for (int q = 0; q < VPL; ++q) {
-      const int e = q * 32 + lane;
-      if (e < E && !((picked >> q) & 1u) && v[q] > bv) {
-        bv = v[q];
-        bi = e;
-      }
+      const int e = expert_of<VEC>(q, lane);
+      key[q] = e < E ? order_key(__ldcs(row + e)) : 0u;
     }
+  }
+  uint32_t my_key = 0u;
+  int my_i = 0;
+  for (int j = 0; j < K; ++j) {
+    uint32_t bk = 0u;
+    int be = 0;
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float ov = __shfl_xor_sync(kFull, bv, off);
-      const int oi = __shfl_xor_sync(kFull, bi, off);
-      if (ov > bv || (ov == bv && oi < bi)) {
-        bv = ov;
-        bi = oi;
+    for (int q = 0; q < VPL; ++q)
+      if (key[q] > bk) {
+        bk = key[q];
+        be = expert_of<VEC>(q, lane);
       }
-    }
-    if (bi == INT_MAX) {
-      // fewer than k finite logits: take the lowest unpicked id, flag it
-      int cand = INT_MAX;
+    const uint32_t m = __reduce_max_sync(kFull, bk);
+    const int e = int(__reduce_min_sync(kFull, bk == m ? uint32_t(be) : 0xFFFFFFFFu));
 #pragma unroll
-      for (int q = VPL - 1; q >= 0; --q) {
-        const int e = q * 32 + lane;
-        if (e < E && !((picked >> q) & 1u)) cand = e;
-      }
-      bi = __reduce_min_sync(kFull, cand);
-      bv = -INFINITY;
-      nonfinite = true;
-    }
-    if ((bi & 31) == lane) picked |= 1u << (bi >> 5);
+    for (int q = 0; q < VPL; ++q)
+      if (expert_of<VEC>(q, lane) == e) key[q] = 0u;
     if (lane == j) {
-      my_v = bv;
-      my_i = bi;
+      my_key = m;
+      my_i = e;
     }
   }
   // softmax over the k winners, shifted by the largest (lane 0's)
-  const float m = __shfl_sync(kFull, my_v, 0);
-  const float ex = lane < K ? expf(my_v - m) : 0.f;
+  const float v = key_value(my_key);
+  const float top = __shfl_sync(kFull, v, 0);
+  const float ex = lane < K ? expf(v - top) : 0.f;
   float s = ex;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(kFull, s, off);
   if (lane < K) {
-    a.topk_idx[int64_t(t) * K + lane] = my_i;
-    a.topk_w[int64_t(t) * K + lane] = ex / s;
-    s_sel[tl * K + lane] = my_i;
+    a.topk_idx[t * K + lane] = my_i;
+    a.topk_w[t * K + lane] = ex / s;
   }
-  if (nonfinite && lane == 0) set_status(a.ws, MOE_ERR_NONFINITE);
+  if (__any_sync(kFull, lane < K && my_key == 1u) && lane == 0) set_status(a.ws, MOE_ERR_NONFINITE);
+  return my_i;
 }
 
-template <int VPL>
-__global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteArgs a) {
-  __shared__ int32_t s_sel[kRouteTokens * kMaxTopK];  // picks of the block's tokens; scan scratch later
-  __shared__ uint32_t s_mask[2 * kMaxExperts];        // [group][expert] token masks; scan scratch later
-  __shared__ int s_last;
+// Phase 2 for column unit u (experts [u*W, u*W + W)).
+template <int W>
+__device__ __forceinline__ void scan_column(const RouteArgs& a, int u, int32_t* s_tot,
+                                            void* s_part_raw, void* s_warp_raw, int32_t* s_off) {
+  using V = typename std::conditional<W == 4, int4, int>::type;
+  V* s_part = static_cast<V*>(s_part_raw);
+  V* s_warp = static_cast<V*>(s_warp_raw);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int B = a.blocks, E = a.E;
+  const int per_rank = E / a.R;
+  const int e0 = u * W;
+  const int lo = (e0 / per_rank) * per_rank, hi = e0 + W;
+  const int64_t row = E / W;  // row stride in column units
+  V zero;
+  if constexpr (W == 4) zero = make_int4(0, 0, 0, 0);
+  else zero = 0;
+  auto add = [](V& x, const V& y) {
+    if constexpr (W == 4) { x.x += y.x; x.y += y.y; x.z += y.z; x.w += y.w; }
+    else x += y;
+  };
+  const V* cnt = reinterpret_cast<const V*>(a.blk);
+  // ---- totals of the experts [lo, hi)
+  if ((lo % W) == 0) {
+    const int u0 = lo / W, nu = (hi - lo) / W;
+    int tpu = kRouteThreads / nu;
+    const int tpu_smem = kMaxSpan / nu;
+    tpu = tpu > tpu_smem ? tpu_smem : tpu;
+    tpu = tpu < 1 ? 1 : (tpu > B ? B : tpu);
+    for (int task = tid; task < nu * tpu; task += kRouteThreads) {
+      const int uu = task % nu, c = task / nu;
+      const int b0 = int(int64_t(B) * c / tpu), b1 = int(int64_t(B) * (c + 1) / tpu);
+      V sum = zero;
+#pragma unroll 8
+      for (int b = b0; b < b1; ++b) add(sum, __ldcg(cnt + int64_t(b) * row + u0 + uu));
+      s_part[task] = sum;
+    }
+    __syncthreads();
+    for (int uu = tid; uu < nu; uu += kRouteThreads) {
+      V sum = zero;
+      for (int c = 0; c < tpu; ++c) add(sum, s_part[c * nu + uu]);
+      if constexpr (W == 4) {
+        s_tot[uu * 4 + 0] = sum.x; s_tot[uu * 4 + 1] = sum.y;
+        s_tot[uu * 4 + 2] = sum.z; s_tot[uu * 4 + 3] = sum.w;
+      } else {
+        s_tot[uu] = sum;
+      }
+    }
+  } else {
+    // a quad that starts inside a rank (E/R not a multiple of 4): per expert
+    for (int e = lo + warp; e < hi; e += kWarps) {
+      int sum = 0;
+      for (int b = lane; b < B; b += 32) sum += __ldcg(a.blk + int64_t(b) * E + e);
+      sum = __reduce_add_sync(kFull, sum);
+      if (lane == 0) s_tot[e - lo] = sum;
+    }
+  }
+  __syncthreads();
+  // ---- offsets of this unit's experts: one warp each
+  if (warp < W) {
+    const int e = e0 + warp;
+    const int r = e / per_rank;
+    int sum = 0;
+    for (int e2 = r * per_rank + lane; e2 < e; e2 += 32) sum += s_tot[e2 - lo];
+    sum = __reduce_add_sync(kFull, sum);
+    if (lane == 0) {
+      const int off = r * a.region_rows + sum;
+      s_off[warp] = off;
+      a.expert_off[e] = off;
+      a.counts[e] = s_tot[e - lo];
+    }
+  }
+  __syncthreads();
+  // ---- exclusive scan of this unit's own columns over the route blocks
+  V* base = reinterpret_cast<V*>(a.bases) + u;
+  const V* own = cnt + u;
+  const int per = (B + kRouteThreads - 1) / kRouteThreads;
+  const int b0 = min(B, tid * per), b1 = min(B, b0 + per);
+  V sum = zero;
+  for (int b = b0; b < b1; ++b) add(sum, __ldcg(own + int64_t(b) * row));
+  V incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    V y;
+    if constexpr (W == 4) {
+      y.x = __shfl_up_sync(kFull, incl.x, o); y.y = __shfl_up_sync(kFull, incl.y, o);
+      y.z = __shfl_up_sync(kFull, incl.z, o); y.w = __shfl_up_sync(kFull, incl.w, o);
+    } else {
+      y = __shfl_up_sync(kFull, incl, o);
+    }
+    if (lane >= o) add(incl, y);
+  }
+  if (lane == 31) s_warp[warp] = incl;
+  __syncthreads();
+  V run;
+  if constexpr (W == 4) run = make_int4(s_off[0], s_off[1], s_off[2], s_off[3]);
+  else run = s_off[0];
+  for (int w = 0; w < warp; ++w) add(run, s_warp[w]);
+  // run + (incl - sum) = absolute base of this thread's first block
+  V ex = incl;
+  if constexpr (W == 4) { ex.x -= sum.x; ex.y -= sum.y; ex.z -= sum.z; ex.w -= sum.w; }
+  else ex -= sum;
+  add(run, ex);
+  for (int b = b0; b < b1; ++b) {
+    base[int64_t(b) * row] = run;
+    add(run, __ldcg(own + int64_t(b) * row));
+  }
+  __syncthreads();  // shared scratch is reused by the next unit
+}
 
+template <int VPL, int VEC>
+__global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(RouteArgs a) {
+  __shared__ int32_t s_sel[kRouteTokens * kMaxTopK];  // picks of the block's tokens
+  __shared__ uint32_t s_mask[kMaxExperts];            // token mask per expert
+  __shared__ int32_t s_tot[kMaxSpan];
+  __shared__ int4 s_part[kMaxSpan];
+  __shared__ int4 s_warp[kWarps];
+  __shared__ int32_t s_off[4];
   const int E = a.E, K = a.K;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int t_base = blockIdx.x * kRouteTokens;
-  const int valid = max(0, min(kRouteTokens, a.n - t_base));
-  for (int i = tid; i < 2 * E; i += kRouteThreads) s_mask[i] = 0;
+  grid_dependency_wait();
 
-  // ---- phase 1: route this warp's tokens, G at a time with their logits prefetched
-  constexpr int G = (32 / VPL) < kTokPerWarp ? (32 / VPL < 1 ? 1 : 32 / VPL) : kTokPerWarp;
-  for (int i0 = 0; i0 < kTokPerWarp; i0 += G) {
-    float v[G][VPL];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const int tl = warp * kTokPerWarp + i0 + g;
-      const float* row = a.logits + int64_t(t_base + tl) * E;
-#pragma unroll
-      for (int q = 0; q < VPL; ++q) {
-        const int e = q * 32 + lane;
-        v[g][q] = (tl < valid && e < E) ? __ldcs(row + e) : -INFINITY;
-      }
+  // ---- phase 1: route blocks b = blockIdx.x, blockIdx.x + grid, ...
+  for (int b = blockIdx.x; b < a.blocks; b += gridDim.x) {
+    const int t_base = b * kRouteTokens;
+    const int valid = max(0, min(kRouteTokens, a.n - t_base));
+    for (int i = tid; i < E; i += kRouteThreads) s_mask[i] = 0;
+    if (warp < valid) {
+      const int e = route_token<VPL, VEC>(a, int64_t(t_base) + warp, lane);
+      if (lane < K) s_sel[warp * K + lane] = e;
     }
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const int tl = warp * kTokPerWarp + i0 + g;
-      if (tl < valid) route_token<VPL>(a, v[g], t_base + tl, tl, lane, s_sel);
+    __syncthreads();
+    for (int p = tid; p < valid * K; p += kRouteThreads)
+      atomicOr(&s_mask[s_sel[p]], 1u << (p / K));
+    __syncthreads();
+    for (int p = tid; p < valid * K; p += kRouteThreads) {
+      const int tl = p / K;
+      a.rank[int64_t(t_base) * K + p] = uint8_t(__popc(s_mask[s_sel[p]] & ((1u << tl) - 1u)));
     }
+    for (int e = tid; e < E; e += kRouteThreads) a.blk[int64_t(b) * E + e] = __popc(s_mask[e]);
+    __syncthreads();
   }
-  __syncthreads();
 
-  // ---- phase 2: group masks -> in-block ranks and block counts
-  for (int p = tid; p < valid * K; p += kRouteThreads) {
-    const int tl = p / K;
-    atomicOr(&s_mask[(tl >> 5) * E + s_sel[p]], 1u << (tl & 31));
-  }
-  __syncthreads();
-  for (int p = tid; p < valid * K; p += kRouteThreads) {
-    const int tl = p / K, e = s_sel[p];
-    int r = __popc(s_mask[(tl >> 5) * E + e] & ((1u << (tl & 31)) - 1u));
-    if (tl >= 32) r += __popc(s_mask[e]);
-    a.rank[int64_t(t_base) * K + p] = uint8_t(r);
-  }
-  for (int e = tid; e < E; e += kRouteThreads)
-    a.blk[int64_t(blockIdx.x) * E + e] = __popc(s_mask[e]) + __popc(s_mask[E + e]);
+  if (!grid_barrier(a.ws, gridDim.x)) return;
 
-  // ---- phase 3: the last block scans the count table
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    Ctrl* c = reinterpret_cast<Ctrl*>(a.ws);
-    const unsigned prev = atomicAdd(&c->ticket, 1u);
-    s_last = (prev == gridDim.x - 1);
+  // ---- phase 2: column units u = blockIdx.x, blockIdx.x + grid, ...
+  if ((E & 3) == 0) {
+    for (int u = blockIdx.x; u < E / 4; u += gridDim.x)
+      scan_column<4>(a, u, s_tot, s_part, s_warp, s_off);
+  } else {
+    for (int u = blockIdx.x; u < E; u += gridDim.x)
+      scan_column<1>(a, u, s_tot, s_part, s_warp, s_off);
   }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
+  if (blockIdx.x == 0 && tid == 0) a.expert_off[E] = a.R * a.region_rows;
+  grid_dependents_launch();
+}
 
-  const int B = gridDim.x;
-  // Column units are 4 experts read as one int4 when E % 4 == 0, else one
-  // expert.  tpc threads split each column unit into tpc chunks of blocks.
-  const bool quad = (E & 3) == 0;
-  const int cols = quad ? E / 4 : E;
-  int tpc = kRouteThreads / cols;
-  tpc = tpc < 1 ? 1 : (tpc > B ? B : tpc);
-  int32_t* s_part = s_sel;                              // [tpc][E] chunk sums -> chunk bases
-  int32_t* s_cnt = reinterpret_cast<int32_t*>(s_mask);  // [E] totals
-  int32_t* s_off = s_cnt + E;                           // [E] expert offsets
-  for (int task = tid; task < cols * tpc; task += kRouteThreads) {
-    const int col = task % cols, c = task / cols;
-    const int b0 = int(int64_t(B) * c / tpc), b1 = int(int64_t(B) * (c + 1) / tpc);
-    if (quad) {
-      int4 sum = make_int4(0, 0, 0, 0);
-#pragma unroll 16
-      for (int b = b0; b < b1; ++b) {
-        const int4 x = __ldcg(reinterpret_cast<const int4*>(a.blk + int64_t(b) * E) + col);
-        sum.x += x.x; sum.y += x.y; sum.z += x.z; sum.w += x.w;
-      }
-      int32_t* dst = s_part + c * E + col * 4;
-      dst[0] = sum.x; dst[1] = sum.y; dst[2] = sum.z; dst[3] = sum.w;
-    } else {
-      int sum = 0;
-#pragma unroll 16
-      for (int b = b0; b < b1; ++b) sum += __ldcg(a.blk + int64_t(b) * E + col);
-      s_part[c * E + col] = sum;
-    }
+// Cooperative launch: every block resident, as the grid barrier requires.
+template <int VPL, int VEC>
+cudaError_t launch_coop(const RouteArgs& a, int sms, cudaStream_t st) {
+  static int per_sm[64] = {0};  // resident blocks per SM, per device
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 64) return cudaErrorInvalidDevice;
+  if (per_sm[dev] == 0) {
+    int nb = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, route_kernel<VPL, VEC>, kRouteThreads, 0);
+    if (e != cudaSuccess) return e;
+    if (nb < 1) return cudaErrorInvalidConfiguration;
+    per_sm[dev] = nb;
   }
-  __syncthreads();
-  for (int e = tid; e < E; e += kRouteThreads) {
-    int run = 0;
-    for (int c = 0; c < tpc; ++c) {
-      const int x = s_part[c * E + e];
-      s_part[c * E + e] = run;
-      run += x;
-    }
-    s_cnt[e] = run;
-    a.counts[e] = run;
-  }
-  __syncthreads();
-  const int per_rank = E / a.R;
-  for (int e = tid; e < E; e += kRouteThreads) {
-    const int r = e / per_rank;
-    int off = r * a.region_rows;
-    for (int e2 = r * per_rank; e2 < e; ++e2) off += s_cnt[e2];
-    s_off[e] = off;
-    a.expert_off[e] = off;
-  }
-  if (tid == 0) a.expert_off[E] = a.R * a.region_rows;
-  __syncthreads();
-  for (int task = tid; task < cols * tpc; task += kRouteThreads) {
-    const int col = task % cols, c = task / cols;
-    const int b0 = int(int64_t(B) * c / tpc), b1 = int(int64_t(B) * (c + 1) / tpc);
-    if (quad) {
-      const int e = col * 4;
-      int4 run = make_int4(s_off[e] + s_part[c * E + e], s_off[e + 1] + s_part[c * E + e + 1],
-                           s_off[e + 2] + s_part[c * E + e + 2], s_off[e + 3] + s_part[c * E + e + 3]);
-#pragma unroll 8
-      for (int b = b0; b < b1; ++b) {
-        int4* p = reinterpret_cast<int4*>(a.blk + int64_t(b) * E) + col;
-        const int4 x = __ldcg(p);
-        *p = run;
-        run.x += x.x; run.y += x.y; run.z += x.z; run.w += x.w;
-      }
-    } else {
-      int run = s_off[col] + s_part[c * E + col];
-#pragma unroll 8
-      for (int b = b0; b < b1; ++b) {
-        int32_t* p = a.blk + int64_t(b) * E + col;
-        const int x = __ldcg(p);
-        *p = run;
-        run += x;
-      }
-    }
-  }
-  if (tid == 0) reinterpret_cast<Ctrl*>(a.ws)->ticket = 0u;
+  const int cols = (a.E & 3) == 0 ? a.E / 4 : a.E;
+  int grid = a.blocks > cols ? a.blocks : cols;
+  if (grid > per_sm[dev] * sms) grid = per_sm[dev] * sms;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(grid));
+  cfg.blockDim = dim3(kRouteThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, route_kernel<VPL, VEC>, a);
 }
 
 }  // namespace
@@ -253,28 +329,38 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteArgs a) {
 cudaError_t launch_route(const moe_plan& p, int32_t n, const float* logits, int32_t* topk_idx,
                          float* topk_w, int32_t* counts, int32_t* expert_off, void* ws,
                          cudaStream_t st) {
+  char* w = static_cast<char*>(ws);
   RouteArgs a;
   a.logits = logits;
   a.topk_idx = topk_idx;
   a.topk_w = topk_w;
   a.counts = counts;
   a.expert_off = expert_off;
-  a.blk = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + p.lay.blk);
-  a.rank = reinterpret_cast<uint8_t*>(static_cast<char*>(ws) + p.lay.rank);
+  a.blk = reinterpret_cast<int32_t*>(w + p.lay.blk);
+  a.bases = reinterpret_cast<int32_t*>(w + p.lay.bases);
+  a.rank = reinterpret_cast<uint8_t*>(w + p.lay.rank);
   a.ws = ws;
   a.n = n;
   a.E = p.d.n_experts;
   a.K = p.d.top_k;
   a.R = p.d.n_ranks;
+  a.blocks = route_blocks(n);
   a.region_rows = int32_t(region_rows(p, n));
-  const dim3 grid(route_blocks(n)), block(kRouteThreads);
-  const int vpl = (a.E + 31) / 32;
-  if (vpl <= 1) route_kernel<1><<<grid, block, 0, st>>>(a);
-  else if (vpl <= 2) route_kernel<2><<<grid, block, 0, st>>>(a);
-  else if (vpl <= 4) route_kernel<4><<<grid, block, 0, st>>>(a);
-  else if (vpl <= 8) route_kernel<8><<<grid, block, 0, st>>>(a);
-  else route_kernel<16><<<grid, block, 0, st>>>(a);
-  return cudaGetLastError();
+  const int sms = num_sms();
+  const int E = a.E;
+  if (E % 128 == 0) {
+    // float4 layout: E / 32 values per lane, a multiple of 4
+    if (E == 128) return launch_coop<4, 4>(a, sms, st);
+    if (E == 256) return launch_coop<8, 4>(a, sms, st);
+    if (E == 384) return launch_coop<12, 4>(a, sms, st);
+    return launch_coop<16, 4>(a, sms, st);
+  }
+  const int vpl = (E + 31) / 32;
+  if (vpl <= 1) return launch_coop<1, 1>(a, sms, st);
+  if (vpl <= 2) return launch_coop<2, 1>(a, sms, st);
+  if (vpl <= 4) return launch_coop<4, 1>(a, sms, st);
+  if (vpl <= 8) return launch_coop<8, 1>(a, sms, st);
+  return launch_coop<16, 1>(a, sms, st);
 }
 
 }  // namespace moe
