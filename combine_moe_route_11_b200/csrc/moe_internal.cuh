@@ -69,6 +69,9 @@ cudaError_t set_smem_limit(const void* kernel, int bytes);
 cudaError_t launch_route(const moe_plan& p, int32_t n, const float* logits, int32_t* topk_idx,
                          float* topk_w, int32_t* counts, int32_t* expert_off, void* ws,
                          cudaStream_t st);
+cudaError_t launch_route_on(const moe_plan& p, int32_t n, const float* logits, int32_t* topk_idx,
+                            float* topk_w, int32_t* counts, int32_t* expert_off, void* ctrl,
+                            int32_t* blk, int32_t* bases, uint8_t* rank, cudaStream_t st);
 cudaError_t launch_dispatch(const moe_plan& p, int32_t n, const void* x, const float* x_scale,
                             const int32_t* topk_idx, void* recv, float* recv_scale,
                             int32_t* slot_of, int32_t* src_of, void* ws, cudaStream_t st);

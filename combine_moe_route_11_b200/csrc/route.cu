@@ -364,3 +364,44 @@ cudaError_t launch_route(const moe_plan& p, int32_t n, const float* logits, int3
 }
 
 }  // namespace moe
+
+namespace moe {
+
+// The route kernels on caller-chosen scratch: ctrl (control words), blk and
+// bases ([route blocks, E] int32 each) and rank ([n, k] bytes).
+cudaError_t launch_route_on(const moe_plan& p, int32_t n, const float* logits, int32_t* topk_idx,
+                            float* topk_w, int32_t* counts, int32_t* expert_off, void* ctrl,
+                            int32_t* blk, int32_t* bases, uint8_t* rank, cudaStream_t st) {
+  RouteArgs a;
+  a.logits = logits;
+  a.topk_idx = topk_idx;
+  a.topk_w = topk_w;
+  a.counts = counts;
+  a.expert_off = expert_off;
+  a.blk = blk;
+  a.bases = bases;
+  a.rank = rank;
+  a.ws = ctrl;
+  a.n = n;
+  a.E = p.d.n_experts;
+  a.K = p.d.top_k;
+  a.R = p.d.n_ranks;
+  a.blocks = route_blocks(n);
+  a.region_rows = int32_t(region_rows(p, n));
+  const int sms = num_sms();
+  const int E = a.E;
+  if (E % 128 == 0) {
+    if (E == 128) return launch_coop<4, 4>(a, sms, st);
+    if (E == 256) return launch_coop<8, 4>(a, sms, st);
+    if (E == 384) return launch_coop<12, 4>(a, sms, st);
+    return launch_coop<16, 4>(a, sms, st);
+  }
+  const int vpl = (E + 31) / 32;
+  if (vpl <= 1) return launch_coop<1, 1>(a, sms, st);
+  if (vpl <= 2) return launch_coop<2, 1>(a, sms, st);
+  if (vpl <= 4) return launch_coop<4, 1>(a, sms, st);
+  if (vpl <= 8) return launch_coop<8, 1>(a, sms, st);
+  return launch_coop<16, 1>(a, sms, st);
+}
+
+}  // namespace moe

@@ -1,0 +1,71 @@
+// moe_route_topk_noalloc: the routing call for callers that cannot allocate
+// device memory.  Its scratch is a fixed array compiled into this library
+// instead of a caller-provided workspace.
+#include "moe_internal.cuh"
+
+#include <mutex>
+
+namespace {
+
+// Scratch of moe_route_topk_noalloc: the control words, the per-block count
+// and base tables and the per-token ranks of one call.  Every GPU that loads
+// this library holds these bytes until the process exits.
+static __device__ __align__(256) unsigned char g_route_scratch[MOE_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_setup_mutex;
+void* g_scratch_addr[kMaxDevices] = {nullptr};
+
+// Device address of g_route_scratch on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address must come from
+// the runtime, once per device, with that device current.
+cudaError_t scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_setup_mutex);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_route_scratch);
+    if (e != cudaSuccess) return e;
+    if (p == nullptr) return cudaErrorInvalidSymbol;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" MOE_API size_t moe_route_topk_noalloc_bytes(const moe_plan* p, int32_t n) {
+  if (!p || n < 0) return 0;
+  const size_t table = moe::align256(size_t(moe::route_blocks(n)) * p->d.n_experts * 4);
+  return sizeof(moe::Ctrl) + 2 * table + moe::align256(size_t(n) * p->d.top_k);
+}
+
+extern "C" MOE_API moe_status moe_route_topk_noalloc(const moe_plan* p, int32_t n,
+                                                     const float* logits, int32_t* topk_idx,
+                                                     float* topk_w, int32_t* counts,
+                                                     int32_t* expert_off, moe_stream_t stream) {
+  if (!p || n < 0 || n > p->d.n_max) return MOE_ERR_INVALID_ARG;
+  if (!counts || !expert_off || (n > 0 && (!logits || !topk_idx || !topk_w)))
+    return MOE_ERR_INVALID_ARG;
+  if (n > 0 && (reinterpret_cast<uintptr_t>(logits) & 15u)) return MOE_ERR_INVALID_ARG;
+  if (moe_route_topk_noalloc_bytes(p, n) > MOE_NOALLOC_SCRATCH_BYTES) return MOE_ERR_WORKSPACE;
+  void* base = nullptr;
+  if (scratch_address(&base) != cudaSuccess) return MOE_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* b = static_cast<char*>(base);
+  const size_t table = moe::align256(size_t(moe::route_blocks(n)) * p->d.n_experts * 4);
+  int32_t* blk = reinterpret_cast<int32_t*>(b + sizeof(moe::Ctrl));
+  int32_t* bases = reinterpret_cast<int32_t*>(b + sizeof(moe::Ctrl) + table);
+  uint8_t* rank = reinterpret_cast<uint8_t*>(b + sizeof(moe::Ctrl) + 2 * table);
+  // The array keeps whatever the previous call left; the barrier counter and
+  // the status word must start at zero.  The tables are fully rewritten.
+  if (cudaMemsetAsync(b, 0, sizeof(moe::Ctrl), st) != cudaSuccess) return MOE_ERR_CUDA;
+  const cudaError_t e = moe::launch_route_on(*p, n, logits, topk_idx, topk_w, counts, expert_off,
+                                             b, blk, bases, rank, st);
+  if (e == cudaSuccess) return MOE_OK;
+  return e == cudaErrorNotSupported ? MOE_ERR_UNSUPPORTED : MOE_ERR_CUDA;
+}

@@ -203,6 +203,32 @@ MOE_API moe_status moe_get_status(const moe_plan* plan, void* ws, moe_stream_t s
  * it), enqueued on `stream`. */
 MOE_API moe_status moe_workspace_init(const moe_plan* plan, void* ws, moe_stream_t stream);
 
+/* Bytes of the fixed scratch array that moe_route_topk_noalloc uses. */
+#define MOE_NOALLOC_SCRATCH_BYTES (1u << 20)
+
+/* No counterpart in the method's description: a convenience of this library.
+ * The same routing as moe_route_topk (same outputs, same layout) for callers
+ * that cannot allocate device memory for a workspace -- for instance a plugin
+ * whose host framework owns every device allocation and hands out none, or
+ * code that must not allocate once it is running.  Its scratch (control
+ * words, per-block tables, ranks) is one array of MOE_NOALLOC_SCRATCH_BYTES
+ * compiled into this library, which every GPU that loads the library keeps
+ * until the process exits; the call allocates and frees nothing.
+ * moe_route_topk_noalloc_bytes(plan, n) is the scratch a call with n tokens
+ * needs; larger calls return MOE_ERR_WORKSPACE before enqueueing anything.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  All calls on a device share the one array, so calls that overlap
+ * on the GPU (other streams, other host threads) race and corrupt each
+ * other: order them.  Each call clears the words that must start at zero.
+ * Device-detected errors are recorded in the array, where moe_get_status
+ * cannot see them; the per-block tables stay inside the array, so this
+ * call's routing cannot feed moe_dispatch. */
+MOE_API size_t moe_route_topk_noalloc_bytes(const moe_plan* plan, int32_t n);
+MOE_API moe_status moe_route_topk_noalloc(const moe_plan* plan, int32_t n, const float* logits,
+                                          int32_t* topk_idx, float* topk_w, int32_t* counts,
+                                          int32_t* expert_off, moe_stream_t stream);
+
 /* Human-readable name of a status code (static string). */
 MOE_API const char* moe_strerror(moe_status status);
 
