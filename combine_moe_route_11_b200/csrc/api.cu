@@ -118,7 +118,7 @@ moe_status moe_plan_create(const moe_desc* desc, moe_plan** out) {
   if (d.inter < 0) return MOE_ERR_INVALID_ARG;
   if (d.inter > 0) {
     if (d.x_dtype != MOE_BF16 || d.y_dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
-    if (d.hidden % 128 || d.inter % 128) return MOE_ERR_UNSUPPORTED;
+    if (d.hidden % 256 || d.inter % 128) return MOE_ERR_UNSUPPORTED;
   }
   moe_plan tmp;
   tmp.d = d;

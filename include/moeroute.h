@@ -109,7 +109,7 @@ typedef struct moe_plan moe_plan;
 /* Validate `desc` and build a plan (host only, no CUDA call).
  * Requires: every row (x, Y, out) a multiple of 16 bytes; scale_block > 0
  * only with FP8 rows and dividing D; T(n_max) < 2^31; for inter > 0 also
- * x = y = BF16, D % 128 == 0 and I % 128 == 0.  *out is set only on MOE_OK. */
+ * x = y = BF16, D % 256 == 0 and I % 128 == 0.  *out is set only on MOE_OK. */
 MOE_API moe_status moe_plan_create(const moe_desc* desc, moe_plan** out);
 MOE_API void moe_plan_destroy(moe_plan* plan);
 
