@@ -72,6 +72,22 @@ def describe(cfg, n: int) -> str:
     return s
 
 
+def step_config(cfg, n: int, n_sets: int, world: int) -> dict:
+    """The `config` object shared by both arms' JSON lines."""
+    step_bytes = algorithmic_bytes(cfg, n)["step"]
+    return {"workload": describe(cfg, n), "parallelism": f"replicas{world}",
+            "l2": (f"no flush: {n_sets} buffer set(s) rotate so a step's data was last touched "
+                   f">= 4x L2 ({step_bytes * max(1, n_sets - 1) / 1e6:.0f} MB of traffic) "
+                   f"earlier; steps run back to back"),
+            "timed": "route(top-k+counts+scan) + dispatch + combine, 3 launches/step",
+            "y_source": "identity expert output, produced once before timing"}
+
+
+def buffer_sets(cfg, n: int) -> int:
+    step = algorithmic_bytes(cfg, n)["step"]
+    return 1 if step >= 4 * L2_BYTES else max(1, min(32, -(-4 * L2_BYTES // step) + 1))
+
+
 def read_peaks() -> tuple[float, str]:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -243,7 +259,7 @@ def run_reference(args, cfg):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt / args.steps * 1e3 * cfg.n / n, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": describe(cfg, cfg.n)},
+            "config": step_config(cfg, cfg.n, buffer_sets(cfg, cfg.n), args.gpus),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -263,7 +279,7 @@ def run_ours(args, cfg):
     nb = algorithmic_bytes(cfg, n)
     # Buffer sets rotate so that a step never finds its data in L2: the other
     # sets' traffic between two uses of a set is at least 4x the L2 size.
-    n_sets = max(1, min(32, -(-4 * L2_BYTES // nb["step"]) + 1)) if nb["step"] < 4 * L2_BYTES else 1
+    n_sets = buffer_sets(cfg, n)
     sets = []
     for si in range(n_sets):
         inp = workloads.make_inputs(cfg, seed=rank * 1000 + si, n=n)
@@ -415,12 +431,7 @@ def run_ours(args, cfg):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic",
-            "config": {"workload": describe(cfg, n), "parallelism": f"replicas{world}",
-                       "l2": (f"no flush: {n_sets} buffer set(s) rotate so a step's data "
-                              f"was last touched >= 4x L2 ({nb['step'] * max(1, n_sets - 1) / 1e6:.0f}"
-                              f" MB of traffic) earlier; steps run back to back"),
-                       "timed": "route(top-k+counts+scan) + dispatch + combine, 3 launches/step",
-                       "y_source": "identity expert output, produced once before timing"},
+            "config": step_config(cfg, n, n_sets, world),
             "hbm_gbs": step_gbs, "hbm_pct_of_peak": 100.0 * step_gbs / peak,
             "kernel_us": {k: v * 1e3 for k, v in kern_ms.items()},
             "algorithmic_bytes": nb,
