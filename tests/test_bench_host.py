@@ -1,0 +1,67 @@
+"""Host-side logic of bench.py without a GPU: max-over-ranks timing and the
+whole-job aggregate across two gloo ranks, the algorithmic byte counts, and
+the buffer-set rotation that keeps steps out of L2."""
+import os
+import socket
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import torch
+    import bench
+    w, r, _ = bench.init_dist()
+    dev = torch.device("cpu")
+    bench.barrier(dev)
+    # rank r "took" 10 + 5r ms per step; the job is as slow as its slowest rank
+    t = bench.reduce_max(10.0 + 5.0 * r, dev)
+    value = bench.job_throughput(w, 4096, t)
+    bench.barrier(dev)
+    import torch.distributed as dist
+    dist.destroy_process_group()
+    q.put((r, w, t, value))
+
+
+def test_two_gloo_ranks_report_the_slowest_rank():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    got = sorted(q.get(timeout=10) for _ in range(world))
+    for r, w, t, value in got:
+        assert w == world
+        assert t == 15.0  # max over ranks
+        assert value == pytest.approx(2 * 4096 / 0.015)
+
+
+def test_algorithmic_bytes_and_rotation():
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads
+    b = bench.algorithmic_bytes(workloads.CONFIGS["prefill"], 4096)
+    assert b["step"] == 805961728
+    assert b["combine"] == 4096 * 8 * 7168 * 2 + 4096 * 8 * 8 + 4096 * 7168 * 2
+    # a prefill step streams > 4x L2 on its own; a decode step needs rotation
+    assert bench.buffer_sets(workloads.CONFIGS["prefill"], 4096) == 1
+    nd = bench.buffer_sets(workloads.CONFIGS["decode"], 128)
+    step = bench.algorithmic_bytes(workloads.CONFIGS["decode"], 128)["step"]
+    assert (nd - 1) * step >= 4 * bench.L2_BYTES
