@@ -72,10 +72,11 @@ def describe(cfg, n: int) -> str:
     return s
 
 
-def step_config(cfg, n: int, n_sets: int, world: int) -> dict:
+def step_config(cfg, n: int, n_sets: int, world: int, graph: bool = False) -> dict:
     """The `config` object shared by both arms' JSON lines."""
     step_bytes = algorithmic_bytes(cfg, n)["step"]
     return {"workload": describe(cfg, n), "parallelism": f"replicas{world}",
+            "launch": "one CUDA graph per step, replayed" if graph else "eager stream launches",
             "l2": (f"no flush: {n_sets} buffer set(s) rotate so a step's data was last touched "
                    f">= 4x L2 ({step_bytes * max(1, n_sets - 1) / 1e6:.0f} MB of traffic) "
                    f"earlier; steps run back to back"),
@@ -293,19 +294,22 @@ def run_ours(args, cfg):
               "ws": plan.new_workspace(dev), "b": plan.new_buffers(n, dev)}
         sets.append(st)
 
+    def cur():
+        return torch.cuda.current_stream(dev)
+
     def route(st):
         b = st["b"]
         mr.moe_route_topk(plan, st["logits"], b["topk_idx"], b["topk_w"], b["counts"],
-                          b["expert_off"], st["ws"], stream)
+                          b["expert_off"], st["ws"], cur())
 
     def dispatch(st):
         b = st["b"]
         mr.moe_dispatch(plan, st["x"], st["xs"], b["topk_idx"], b["recv"], b["recv_scale"],
-                        b["slot_of"], b["src_of"], st["ws"], stream)
+                        b["slot_of"], b["src_of"], st["ws"], cur())
 
     def combine(st):
         b = st["b"]
-        mr.moe_combine(plan, st["y"], b["topk_w"], b["slot_of"], b["out"], st["ws"], stream)
+        mr.moe_combine(plan, st["y"], b["topk_w"], b["slot_of"], b["out"], st["ws"], cur())
 
     # expert output read by combine: identity expert, produced once per set
     for st in sets:
@@ -325,16 +329,16 @@ def run_ours(args, cfg):
 
     def step(st, evs=None):
         if evs:
-            evs[0].record(stream)
+            evs[0].record(cur())
         route(st)
         if evs:
-            evs[1].record(stream)
+            evs[1].record(cur())
         dispatch(st)
         if evs:
-            evs[2].record(stream)
+            evs[2].record(cur())
         combine(st)
         if evs:
-            evs[3].record(stream)
+            evs[3].record(cur())
 
     for i in range(args.warmup):
         step(sets[i % n_sets])
@@ -356,13 +360,27 @@ def run_ours(args, cfg):
     sampler.wait_first()
     for i in range(args.warmup):
         step(sets[i % n_sets])
+    graphs = None
+    if args.graph:
+        # one CUDA graph per buffer set holding one whole step; replayed K times
+        graphs = []
+        for st in sets:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                step(st)
+            graphs.append(g)
+        for i in range(args.warmup):
+            graphs[i % n_sets].replay()
     r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(dev)
     torch.cuda.synchronize(dev)
     t_start = time.time()
     r0.record(stream)
     for i in range(args.steps):
-        step(sets[i % n_sets])
+        if graphs:
+            graphs[i % n_sets].replay()
+        else:
+            step(sets[i % n_sets])
     r1.record(stream)
     torch.cuda.synchronize(dev)
     t_end = time.time()
@@ -436,7 +454,7 @@ def run_ours(args, cfg):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic",
-            "config": step_config(cfg, n, n_sets, world),
+            "config": step_config(cfg, n, n_sets, world, args.graph),
             "hbm_gbs": step_gbs, "hbm_pct_of_peak": 100.0 * step_gbs / peak,
             "kernel_us": {k: v * 1e3 for k, v in kern_ms.items()},
             "algorithmic_bytes": nb,
@@ -571,6 +589,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", action="store_true",
+                    help="replay each step as one captured CUDA graph")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override N (smaller batches for profiler captures only)")
     ap.add_argument("--experts", type=int, default=0,

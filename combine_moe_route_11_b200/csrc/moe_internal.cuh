@@ -38,7 +38,7 @@ inline int elem_bytes(int dtype) {
 
 // Byte offsets of every buffer inside a workspace, fixed by n_max.
 struct Layout {
-  size_t ctrl, blk, bases, rank, route_end;
+  size_t ctrl, blk, bases, totals, rank, route_end;
   size_t topk_idx, topk_w, counts, expert_off, slot_of, src_of, recv, recv_scale, y, h, end;
 };
 
@@ -71,7 +71,8 @@ cudaError_t launch_route(const moe_plan& p, int32_t n, const float* logits, int3
                          cudaStream_t st);
 cudaError_t launch_route_on(const moe_plan& p, int32_t n, const float* logits, int32_t* topk_idx,
                             float* topk_w, int32_t* counts, int32_t* expert_off, void* ctrl,
-                            int32_t* blk, int32_t* bases, uint8_t* rank, cudaStream_t st);
+                            int32_t* blk, int32_t* bases, int32_t* totals, uint8_t* rank,
+                            cudaStream_t st);
 cudaError_t launch_dispatch(const moe_plan& p, int32_t n, const void* x, const float* x_scale,
                             const int32_t* topk_idx, void* recv, float* recv_scale,
                             int32_t* slot_of, int32_t* src_of, void* ws, cudaStream_t st);
@@ -122,35 +123,48 @@ __device__ __forceinline__ void set_status(void* ws, int code) {
   atomicCAS(&c->status, 0, code);
 }
 
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_relaxed_gpu(unsigned* p, unsigned v) {
+  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void fence_acq_rel_gpu() {
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
+
 // Barrier across all `blocks` blocks of a grid whose blocks are all resident
-// (cooperative launch).  The wait is bounded (~2^31 cycles); on timeout it
-// records MOE_ERR_TIMEOUT and returns false, and the workspace must be
-// re-initialised before its next use.
+// (cooperative launch).  The block barrier orders the block's writes before
+// thread 0's release fence and arrival; the last arrival bumps the
+// generation, which the others poll with acquire loads.  The wait is bounded
+// (~2^31 cycles); on timeout it records MOE_ERR_TIMEOUT and returns false,
+// and the workspace must be re-initialised before its next use.
 __device__ __forceinline__ bool grid_barrier(void* ws, unsigned blocks) {
   __shared__ int s_ok;
   Ctrl* c = reinterpret_cast<Ctrl*>(ws);
   __syncthreads();
   if (threadIdx.x == 0) {
     bool ok = true;
-    __threadfence();
-    const unsigned gen = *reinterpret_cast<volatile unsigned*>(&c->gen);
-    __threadfence();
+    const unsigned gen = ld_acquire_gpu(&c->gen);
+    fence_acq_rel_gpu();
     if (atomicAdd(&c->arrive, 1u) + 1u == blocks) {
-      atomicExch(&c->arrive, 0u);
-      __threadfence();
+      st_relaxed_gpu(&c->arrive, 0u);
+      fence_acq_rel_gpu();
       atomicAdd(&c->gen, 1u);
     } else {
       const long long t0 = clock64();
-      while (*reinterpret_cast<volatile unsigned*>(&c->gen) == gen) {
+      while (ld_acquire_gpu(&c->gen) == gen) {
         if (clock64() - t0 > (1ll << 31)) {
           ok = false;
           set_status(ws, MOE_ERR_TIMEOUT);
           break;
         }
-        __nanosleep(32);
       }
     }
-    __threadfence();
     s_ok = ok;
   }
   __syncthreads();

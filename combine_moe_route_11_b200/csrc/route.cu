@@ -19,10 +19,12 @@
 //     of the block's tokens that picked it gives each (token, expert) pair
 //     its rank among the block's tokens (popcount of the lower lanes) and the
 //     block's count of the expert;
-//  2. per column of (up to) 4 experts: the count columns of the experts of
-//     its rank below its own give the rank-major offsets, and an exclusive
-//     scan of its own columns over the route blocks gives each block's
-//     absolute base slot (a separate table: other blocks still read counts).
+//     Each block also adds its counts into the expert totals (integer
+//     atomics: the sum does not depend on their order);
+//  2. per column of (up to) 4 experts: the totals of the experts of its rank
+//     below its own give the rank-major offsets, and an exclusive scan of its
+//     own count columns over the route blocks gives each block's absolute
+//     base slot.
 // A slot is then base[block][e] + rank.  All integer results are
 // deterministic: no atomic decides an order.
 #include "moe_internal.cuh"
@@ -37,7 +39,6 @@ namespace {
 
 constexpr unsigned kFull = 0xFFFFFFFFu;
 constexpr int kWarps = kRouteThreads / 32;
-constexpr int kMaxSpan = kMaxExperts + 4;
 
 struct RouteArgs {
   const float* logits;
@@ -47,6 +48,7 @@ struct RouteArgs {
   int32_t* expert_off;
   int32_t* blk;    // [blocks, E] per-block counts
   int32_t* bases;  // [blocks, E] per-block absolute base slots
+  int32_t* totals; // [2, E] expert totals, the half of this call chosen by barrier parity
   uint8_t* rank;   // [n, k]: rank of (t, j) among the block's tokens picking e
   void* ws;
   int32_t n, E, K, R;
@@ -101,25 +103,49 @@ __device__ __forceinline__ int route_token(const RouteArgs& a, int64_t t, int la
       key[q] = e < E ? order_key(__ldcs(row + e)) : 0u;
     }
   }
+  // This lane's best two untaken values (strict compares keep the lower id
+  // first among equal keys).  Each round the warp takes the largest head;
+  // the owning lane moves its second value up, and rescans only when both
+  // were taken -- rare, since the k winners spread over 32 lanes.
+  uint32_t k1 = 0u, k2 = 0u, taken = 0u;
+  int q1 = 0, q2 = 0;
+#pragma unroll
+  for (int q = 0; q < VPL; ++q) {
+    const uint32_t v = key[q];
+    if (v > k1) {
+      k2 = k1; q2 = q1; k1 = v; q1 = q;
+    } else if (v > k2) {
+      k2 = v; q2 = q;
+    }
+  }
+  bool have2 = true;
   uint32_t my_key = 0u;
   int my_i = 0;
   for (int j = 0; j < K; ++j) {
-    uint32_t bk = 0u;
-    int be = 0;
-#pragma unroll
-    for (int q = 0; q < VPL; ++q)
-      if (key[q] > bk) {
-        bk = key[q];
-        be = expert_of<VEC>(q, lane);
-      }
-    const uint32_t m = __reduce_max_sync(kFull, bk);
-    const int e = int(__reduce_min_sync(kFull, bk == m ? uint32_t(be) : 0xFFFFFFFFu));
-#pragma unroll
-    for (int q = 0; q < VPL; ++q)
-      if (expert_of<VEC>(q, lane) == e) key[q] = 0u;
+    const uint32_t m = __reduce_max_sync(kFull, k1);
+    const int e1 = expert_of<VEC>(q1, lane);
+    const int e = int(__reduce_min_sync(kFull, k1 == m ? uint32_t(e1) : 0xFFFFFFFFu));
     if (lane == j) {
       my_key = m;
       my_i = e;
+    }
+    if (k1 == m && e1 == e) {
+      taken |= 1u << q1;
+      if (have2) {
+        k1 = k2; q1 = q2; have2 = false;
+      } else {
+        k1 = k2 = 0u; q1 = q2 = 0;
+#pragma unroll
+        for (int q = 0; q < VPL; ++q) {
+          const uint32_t v = ((taken >> q) & 1u) ? 0u : key[q];
+          if (v > k1) {
+            k2 = k1; q2 = q1; k1 = v; q1 = q;
+          } else if (v > k2) {
+            k2 = v; q2 = q;
+          }
+        }
+        have2 = true;
+      }
     }
   }
   // softmax over the k winners, shifted by the largest (lane 0's)
@@ -137,18 +163,18 @@ __device__ __forceinline__ int route_token(const RouteArgs& a, int64_t t, int la
   return my_i;
 }
 
-// Phase 2 for column unit u (experts [u*W, u*W + W)).
+// Phase 2 for column unit u (experts [u*W, u*W + W)): rank-major offsets
+// from the expert totals, then the exclusive scan of the unit's count columns
+// over the route blocks into absolute bases.
 template <int W>
-__device__ __forceinline__ void scan_column(const RouteArgs& a, int u, int32_t* s_tot,
-                                            void* s_part_raw, void* s_warp_raw, int32_t* s_off) {
+__device__ __forceinline__ void scan_column(const RouteArgs& a, int u, const int32_t* tot,
+                                            void* s_warp_raw, int32_t* s_off) {
   using V = typename std::conditional<W == 4, int4, int>::type;
-  V* s_part = static_cast<V*>(s_part_raw);
   V* s_warp = static_cast<V*>(s_warp_raw);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int B = a.blocks, E = a.E;
   const int per_rank = E / a.R;
   const int e0 = u * W;
-  const int lo = (e0 / per_rank) * per_rank, hi = e0 + W;
   const int64_t row = E / W;  // row stride in column units
   V zero;
   if constexpr (W == 4) zero = make_int4(0, 0, 0, 0);
@@ -158,54 +184,18 @@ __device__ __forceinline__ void scan_column(const RouteArgs& a, int u, int32_t* 
     else x += y;
   };
   const V* cnt = reinterpret_cast<const V*>(a.blk);
-  // ---- totals of the experts [lo, hi)
-  if ((lo % W) == 0) {
-    const int u0 = lo / W, nu = (hi - lo) / W;
-    int tpu = kRouteThreads / nu;
-    const int tpu_smem = kMaxSpan / nu;
-    tpu = tpu > tpu_smem ? tpu_smem : tpu;
-    tpu = tpu < 1 ? 1 : (tpu > B ? B : tpu);
-    for (int task = tid; task < nu * tpu; task += kRouteThreads) {
-      const int uu = task % nu, c = task / nu;
-      const int b0 = int(int64_t(B) * c / tpu), b1 = int(int64_t(B) * (c + 1) / tpu);
-      V sum = zero;
-#pragma unroll 8
-      for (int b = b0; b < b1; ++b) add(sum, __ldcg(cnt + int64_t(b) * row + u0 + uu));
-      s_part[task] = sum;
-    }
-    __syncthreads();
-    for (int uu = tid; uu < nu; uu += kRouteThreads) {
-      V sum = zero;
-      for (int c = 0; c < tpu; ++c) add(sum, s_part[c * nu + uu]);
-      if constexpr (W == 4) {
-        s_tot[uu * 4 + 0] = sum.x; s_tot[uu * 4 + 1] = sum.y;
-        s_tot[uu * 4 + 2] = sum.z; s_tot[uu * 4 + 3] = sum.w;
-      } else {
-        s_tot[uu] = sum;
-      }
-    }
-  } else {
-    // a quad that starts inside a rank (E/R not a multiple of 4): per expert
-    for (int e = lo + warp; e < hi; e += kWarps) {
-      int sum = 0;
-      for (int b = lane; b < B; b += 32) sum += __ldcg(a.blk + int64_t(b) * E + e);
-      sum = __reduce_add_sync(kFull, sum);
-      if (lane == 0) s_tot[e - lo] = sum;
-    }
-  }
-  __syncthreads();
-  // ---- offsets of this unit's experts: one warp each
+  // ---- offsets of this unit's experts from the phase-1 totals: one warp each
   if (warp < W) {
     const int e = e0 + warp;
     const int r = e / per_rank;
     int sum = 0;
-    for (int e2 = r * per_rank + lane; e2 < e; e2 += 32) sum += s_tot[e2 - lo];
+    for (int e2 = r * per_rank + lane; e2 < e; e2 += 32) sum += __ldcg(tot + e2);
     sum = __reduce_add_sync(kFull, sum);
     if (lane == 0) {
       const int off = r * a.region_rows + sum;
       s_off[warp] = off;
       a.expert_off[e] = off;
-      a.counts[e] = s_tot[e - lo];
+      a.counts[e] = __ldcg(tot + e);
     }
   }
   __syncthreads();
@@ -250,13 +240,17 @@ template <int VPL, int VEC>
 __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(RouteArgs a) {
   __shared__ int32_t s_sel[kRouteTokens * kMaxTopK];  // picks of the block's tokens
   __shared__ uint32_t s_mask[kMaxExperts];            // token mask per expert
-  __shared__ int32_t s_tot[kMaxSpan];
-  __shared__ int4 s_part[kMaxSpan];
   __shared__ int4 s_warp[kWarps];
   __shared__ int32_t s_off[4];
+  __shared__ unsigned s_parity;
   const int E = a.E, K = a.K;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   grid_dependency_wait();
+  // This call's half of the totals: the barrier generation's parity, read
+  // before any block can reach the barrier that bumps it.
+  if (tid == 0) s_parity = ld_acquire_gpu(&reinterpret_cast<Ctrl*>(a.ws)->gen) & 1u;
+  __syncthreads();
+  int32_t* tot = a.totals + size_t(s_parity) * E;
 
   // ---- phase 1: route blocks b = blockIdx.x, blockIdx.x + grid, ...
   for (int b = blockIdx.x; b < a.blocks; b += gridDim.x) {
@@ -275,7 +269,11 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(RouteArgs a) {
       const int tl = p / K;
       a.rank[int64_t(t_base) * K + p] = uint8_t(__popc(s_mask[s_sel[p]] & ((1u << tl) - 1u)));
     }
-    for (int e = tid; e < E; e += kRouteThreads) a.blk[int64_t(b) * E + e] = __popc(s_mask[e]);
+    for (int e = tid; e < E; e += kRouteThreads) {
+      const int c = __popc(s_mask[e]);
+      a.blk[int64_t(b) * E + e] = c;
+      if (c) atomicAdd(tot + e, c);  // integer sums: the order does not matter
+    }
     __syncthreads();
   }
 
@@ -283,13 +281,16 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(RouteArgs a) {
 
   // ---- phase 2: column units u = blockIdx.x, blockIdx.x + grid, ...
   if ((E & 3) == 0) {
-    for (int u = blockIdx.x; u < E / 4; u += gridDim.x)
-      scan_column<4>(a, u, s_tot, s_part, s_warp, s_off);
+    for (int u = blockIdx.x; u < E / 4; u += gridDim.x) scan_column<4>(a, u, tot, s_warp, s_off);
   } else {
-    for (int u = blockIdx.x; u < E; u += gridDim.x)
-      scan_column<1>(a, u, s_tot, s_part, s_warp, s_off);
+    for (int u = blockIdx.x; u < E; u += gridDim.x) scan_column<1>(a, u, tot, s_warp, s_off);
   }
-  if (blockIdx.x == 0 && tid == 0) a.expert_off[E] = a.R * a.region_rows;
+  if (blockIdx.x == 0) {
+    // the other half starts the next call at zero
+    int32_t* next = a.totals + size_t(s_parity ^ 1u) * E;
+    for (int e = tid; e < E; e += kRouteThreads) next[e] = 0;
+    if (tid == 0) a.expert_off[E] = a.R * a.region_rows;
+  }
   grid_dependents_launch();
 }
 
@@ -338,6 +339,7 @@ cudaError_t launch_route(const moe_plan& p, int32_t n, const float* logits, int3
   a.expert_off = expert_off;
   a.blk = reinterpret_cast<int32_t*>(w + p.lay.blk);
   a.bases = reinterpret_cast<int32_t*>(w + p.lay.bases);
+  a.totals = reinterpret_cast<int32_t*>(w + p.lay.totals);
   a.rank = reinterpret_cast<uint8_t*>(w + p.lay.rank);
   a.ws = ws;
   a.n = n;
@@ -368,10 +370,12 @@ cudaError_t launch_route(const moe_plan& p, int32_t n, const float* logits, int3
 namespace moe {
 
 // The route kernels on caller-chosen scratch: ctrl (control words), blk and
-// bases ([route blocks, E] int32 each) and rank ([n, k] bytes).
+// bases ([route blocks, E] int32 each), totals ([2, E] int32, zero before the
+// first call) and rank ([n, k] bytes).
 cudaError_t launch_route_on(const moe_plan& p, int32_t n, const float* logits, int32_t* topk_idx,
                             float* topk_w, int32_t* counts, int32_t* expert_off, void* ctrl,
-                            int32_t* blk, int32_t* bases, uint8_t* rank, cudaStream_t st) {
+                            int32_t* blk, int32_t* bases, int32_t* totals, uint8_t* rank,
+                            cudaStream_t st) {
   RouteArgs a;
   a.logits = logits;
   a.topk_idx = topk_idx;
@@ -380,6 +384,7 @@ cudaError_t launch_route_on(const moe_plan& p, int32_t n, const float* logits, i
   a.expert_off = expert_off;
   a.blk = blk;
   a.bases = bases;
+  a.totals = totals;
   a.rank = rank;
   a.ws = ctrl;
   a.n = n;

@@ -41,7 +41,8 @@ cudaError_t scratch_address(void** out) {
 extern "C" MOE_API size_t moe_route_topk_noalloc_bytes(const moe_plan* p, int32_t n) {
   if (!p || n < 0) return 0;
   const size_t table = moe::align256(size_t(moe::route_blocks(n)) * p->d.n_experts * 4);
-  return sizeof(moe::Ctrl) + 2 * table + moe::align256(size_t(n) * p->d.top_k);
+  const size_t totals = moe::align256(size_t(2) * p->d.n_experts * 4);
+  return sizeof(moe::Ctrl) + totals + 2 * table + moe::align256(size_t(n) * p->d.top_k);
 }
 
 extern "C" MOE_API moe_status moe_route_topk_noalloc(const moe_plan* p, int32_t n,
@@ -58,14 +59,17 @@ extern "C" MOE_API moe_status moe_route_topk_noalloc(const moe_plan* p, int32_t 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   char* b = static_cast<char*>(base);
   const size_t table = moe::align256(size_t(moe::route_blocks(n)) * p->d.n_experts * 4);
-  int32_t* blk = reinterpret_cast<int32_t*>(b + sizeof(moe::Ctrl));
-  int32_t* bases = reinterpret_cast<int32_t*>(b + sizeof(moe::Ctrl) + table);
-  uint8_t* rank = reinterpret_cast<uint8_t*>(b + sizeof(moe::Ctrl) + 2 * table);
-  // The array keeps whatever the previous call left; the barrier counter and
-  // the status word must start at zero.  The tables are fully rewritten.
-  if (cudaMemsetAsync(b, 0, sizeof(moe::Ctrl), st) != cudaSuccess) return MOE_ERR_CUDA;
+  const size_t totals_bytes = moe::align256(size_t(2) * p->d.n_experts * 4);
+  int32_t* totals = reinterpret_cast<int32_t*>(b + sizeof(moe::Ctrl));
+  int32_t* blk = reinterpret_cast<int32_t*>(b + sizeof(moe::Ctrl) + totals_bytes);
+  int32_t* bases = reinterpret_cast<int32_t*>(b + sizeof(moe::Ctrl) + totals_bytes + table);
+  uint8_t* rank = reinterpret_cast<uint8_t*>(b + sizeof(moe::Ctrl) + totals_bytes + 2 * table);
+  // The array keeps whatever the previous call left; the control words and
+  // the expert totals must start at zero.  The tables are fully rewritten.
+  if (cudaMemsetAsync(b, 0, sizeof(moe::Ctrl) + totals_bytes, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
   const cudaError_t e = moe::launch_route_on(*p, n, logits, topk_idx, topk_w, counts, expert_off,
-                                             b, blk, bases, rank, st);
+                                             b, blk, bases, totals, rank, st);
   if (e == cudaSuccess) return MOE_OK;
   return e == cudaErrorNotSupported ? MOE_ERR_UNSUPPORTED : MOE_ERR_CUDA;
 }

@@ -199,8 +199,9 @@ MOE_API void* moe_layer_buffer(const moe_plan* plan, void* ws, const char* name)
  * (MOE_ERR_CUDA if the copy itself fails). */
 MOE_API moe_status moe_get_status(const moe_plan* plan, void* ws, moe_stream_t stream);
 
-/* Zero the control words of a workspace (an alternative to zero-filling
- * it), enqueued on `stream`. */
+/* Zero the control words and expert totals of a workspace (an alternative
+ * to zero-filling it), enqueued on `stream`.  Required again after a call
+ * reported MOE_ERR_TIMEOUT. */
 MOE_API moe_status moe_workspace_init(const moe_plan* plan, void* ws, moe_stream_t stream);
 
 /* Bytes of the fixed scratch array that moe_route_topk_noalloc uses. */
