@@ -59,8 +59,8 @@ def algorithmic_bytes(cfg, n: int) -> dict:
     route = n * e * 4 + n * k * 8
     dispatch = n * row + n * k * row + n * k * 8
     combine = n * k * d * yb + n * k * 8 + n * d * ob
-    return {"route": route, "dispatch": dispatch, "combine": combine,
-            "step": route + dispatch + combine}
+    return {"route": route, "dispatch": dispatch, "route_dispatch": route + dispatch,
+            "combine": combine, "step": route + dispatch + combine}
 
 
 def describe(cfg, n: int) -> str:
@@ -307,6 +307,12 @@ def run_ours(args, cfg):
         mr.moe_dispatch(plan, st["x"], st["xs"], b["topk_idx"], b["recv"], b["recv_scale"],
                         b["slot_of"], b["src_of"], st["ws"], cur())
 
+    def route_dispatch(st):
+        b = st["b"]
+        mr.moe_route_dispatch(plan, st["logits"], st["x"], st["xs"], b["topk_idx"], b["topk_w"],
+                              b["counts"], b["expert_off"], b["recv"], b["recv_scale"],
+                              b["slot_of"], b["src_of"], st["ws"], cur())
+
     def combine(st):
         b = st["b"]
         mr.moe_combine(plan, st["y"], b["topk_w"], b["slot_of"], b["out"], st["ws"], cur())
@@ -327,34 +333,34 @@ def run_ours(args, cfg):
         if mr.moe_get_status(plan, st["ws"], stream) != 0:
             raise RuntimeError("device status set before timing")
 
+    # The step is what moe_route_dispatch + moe_combine launch: one fused
+    # route + dispatch kernel for small batches, else the route and dispatch
+    # kernels (the very launches moe_route_dispatch makes at that size).
+    if n <= mr.FUSED_MAX_TOKENS:
+        stages = [("route_dispatch", route_dispatch), ("combine", combine)]
+    else:
+        stages = [("route", route), ("dispatch", dispatch), ("combine", combine)]
+
     def step(st, evs=None):
+        for j, (_, f) in enumerate(stages):
+            if evs:
+                evs[j].record(cur())
+            f(st)
         if evs:
-            evs[0].record(cur())
-        route(st)
-        if evs:
-            evs[1].record(cur())
-        dispatch(st)
-        if evs:
-            evs[2].record(cur())
-        combine(st)
-        if evs:
-            evs[3].record(cur())
+            evs[len(stages)].record(cur())
 
     for i in range(args.warmup):
         step(sets[i % n_sets])
     # pass 1: per-kernel CUDA events inside every step (kernel durations)
     k_steps = min(args.steps, 200)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(k_steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)]
+          for _ in range(k_steps)]
     torch.cuda.synchronize(dev)
     for i in range(k_steps):
         step(sets[i % n_sets], ev[i])
     torch.cuda.synchronize(dev)
-    per = {"route": 0.0, "dispatch": 0.0, "combine": 0.0}
-    for e in ev:
-        per["route"] += e[0].elapsed_time(e[1])
-        per["dispatch"] += e[1].elapsed_time(e[2])
-        per["combine"] += e[2].elapsed_time(e[3])
-    kern_ms = {k: v / k_steps for k, v in per.items()}
+    kern_ms = {name: sum(e[j].elapsed_time(e[j + 1]) for e in ev) / k_steps
+               for j, (name, _) in enumerate(stages)}
     # pass 2: K steps back to back, events only around the region
     sampler = ClockSampler(local)
     sampler.wait_first()
@@ -392,7 +398,7 @@ def run_ours(args, cfg):
     total_ms = reduce_max(r0.elapsed_time(r1), dev)
     ms_step = total_ms / args.steps
     peak, peak_kind = read_peaks()
-    dom = max(("dispatch", "combine"), key=lambda k: kern_ms[k])
+    dom = max((k for k in kern_ms if k != "route"), key=lambda k: kern_ms[k])
     achieved = nb[dom] / (kern_ms[dom] * 1e-3) / 1e9
     step_gbs = nb["step"] / (ms_step * 1e-3) / 1e9
     inp = sets[0]["inp"]
@@ -463,7 +469,7 @@ def run_ours(args, cfg):
                          "traffic": recorded_traffic(cfg.name) if dom == "combine" else None},
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": 3 * args.steps,
+            "gpu_launches": len(stages) * args.steps,
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
@@ -496,13 +502,11 @@ def run_layer(args, cfg):
     ws = plan.new_workspace(dev)
     b = plan.new_buffers(n, dev)
 
-    def route():
-        mr.moe_route_topk(plan, logits, b["topk_idx"], b["topk_w"], b["counts"], b["expert_off"],
-                          ws, stream)
-
-    def dispatch():
-        mr.moe_dispatch(plan, x, None, b["topk_idx"], b["recv"], None, b["slot_of"], b["src_of"],
-                        ws, stream)
+    def route_dispatch():
+        # the call moe_layer makes: one launch at n <= 1024, else two
+        mr.moe_route_dispatch(plan, logits, x, None, b["topk_idx"], b["topk_w"], b["counts"],
+                              b["expert_off"], b["recv"], None, b["slot_of"], b["src_of"], ws,
+                              stream)
 
     def expert():
         mr.moe_expert_swiglu(plan, n, b["recv"], b["counts"], b["expert_off"], wgu, wd, b["h"],
@@ -511,20 +515,21 @@ def run_layer(args, cfg):
     def combine():
         mr.moe_combine(plan, b["y"], b["topk_w"], b["slot_of"], b["out"], ws, stream)
 
-    stages = [route, dispatch, expert, combine]
+    stages = [route_dispatch, expert, combine]
     for _ in range(args.warmup):
         for f in stages:
             f()
     k_steps = min(args.steps, 50)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(k_steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)]
+          for _ in range(k_steps)]
     torch.cuda.synchronize(dev)
     for i in range(k_steps):
         for j, f in enumerate(stages):
             ev[i][j].record(stream)
             f()
-        ev[i][4].record(stream)
+        ev[i][len(stages)].record(stream)
     torch.cuda.synchronize(dev)
-    names = ["route", "dispatch", "expert_gemm", "combine"]
+    names = ["route_dispatch", "expert_gemm", "combine"]
     kern_ms = {nm: sum(e[j].elapsed_time(e[j + 1]) for e in ev) / k_steps
                for j, nm in enumerate(names)}
     sampler = ClockSampler(local)
@@ -587,7 +592,7 @@ def run_layer(args, cfg):
             "roofline_other": other,
             "weight_stream_gbs": wbytes / (kern_ms["expert_gemm"] * 1e-3) / 1e9,
             "weight_stream_frac_of_hbm": wbytes / (kern_ms["expert_gemm"] * 1e-3) / 1e9 / hbm_peak,
-            "gpu_launches": 6 * args.steps,
+            "gpu_launches": (4 if n <= mr.FUSED_MAX_TOKENS else 5) * args.steps,
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)

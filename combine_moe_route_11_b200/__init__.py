@@ -27,6 +27,9 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 DTYPE_CODES = {"f32": 0, "bf16": 1, "fp8_e4m3": 2}
+# Largest batch that moe_route_dispatch runs as one launch (32 route blocks
+# of 32 tokens); larger batches run the route and dispatch kernels.
+FUSED_MAX_TOKENS = 1024
 ELEM_BYTES = {"f32": 4, "bf16": 2, "fp8_e4m3": 1}
 _TORCH = {"f32": (torch.float32,), "bf16": (torch.bfloat16,),
           "fp8_e4m3": (torch.uint8, torch.float8_e4m3fn)}
@@ -49,6 +52,7 @@ _SIGS = {
     "moe_recv_rows": (ctypes.c_int64, [_P, _i32]),
     "moe_route_topk": (ctypes.c_int, [_P, _i32, _P, _P, _P, _P, _P, _P, _P]),
     "moe_dispatch": (ctypes.c_int, [_P, _i32, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_route_dispatch": (ctypes.c_int, [_P, _i32] + [_P] * 13),
     "moe_expert_dequant": (ctypes.c_int, [_P, _i32, _P, _P, _P, _P, _P, _P]),
     "moe_expert_swiglu": (ctypes.c_int, [_P, _i32, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_combine": (ctypes.c_int, [_P, _i32, _P, _P, _P, _P, _P, _P]),
@@ -207,6 +211,30 @@ def moe_dispatch(plan: Plan, x, x_scale, topk_idx, recv, recv_scale, slot_of, sr
     _check(_lib.moe_dispatch(plan.handle, n, _ptr(x), _ptr(x_scale), _ptr(topk_idx), _ptr(recv),
                              _ptr(recv_scale), _ptr(slot_of), _ptr(src_of), _ptr(ws),
                              _stream(stream)), "moe_dispatch")
+
+
+def moe_route_dispatch(plan: Plan, logits, x, x_scale, topk_idx, topk_w, counts, expert_off,
+                       recv, recv_scale, slot_of, src_of, ws, stream=None):
+    """moe_route_topk followed by moe_dispatch; one launch for n <= 1024."""
+    n = logits.shape[0]
+    T = plan.recv_rows(n)
+    _expect(logits, (torch.float32,), (n, plan.n_experts), "logits")
+    _expect(x, _TORCH[plan.x_dtype], (n, plan.hidden), "x")
+    _expect(topk_idx, (torch.int32,), (n, plan.top_k), "topk_idx")
+    _expect(topk_w, (torch.float32,), (n, plan.top_k), "topk_w")
+    _expect(counts, (torch.int32,), (plan.n_experts,), "counts")
+    _expect(expert_off, (torch.int32,), (plan.n_experts + 1,), "expert_off")
+    if recv.shape[0] < T or tuple(recv.shape[1:]) != (plan.hidden,):
+        raise ValueError(f"recv: shape {tuple(recv.shape)}, need at least ({T}, {plan.hidden})")
+    _expect(slot_of, (torch.int32,), (n, plan.top_k), "slot_of")
+    if src_of.shape[0] < T:
+        raise ValueError("src_of too short")
+    if plan.scale_cols:
+        _expect(x_scale, (torch.float32,), (n, plan.scale_cols), "x_scale")
+    _check(_lib.moe_route_dispatch(plan.handle, n, _ptr(logits), _ptr(x), _ptr(x_scale),
+                                   _ptr(topk_idx), _ptr(topk_w), _ptr(counts), _ptr(expert_off),
+                                   _ptr(recv), _ptr(recv_scale), _ptr(slot_of), _ptr(src_of),
+                                   _ptr(ws), _stream(stream)), "moe_route_dispatch")
 
 
 def moe_expert_dequant(plan: Plan, n: int, recv, recv_scale, slot_of, y, ws, stream=None):

@@ -175,6 +175,30 @@ moe_status moe_dispatch(const moe_plan* p, int32_t n, const void* x, const float
                                      src_of, ws, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+moe_status moe_route_dispatch(const moe_plan* p, int32_t n, const float* logits, const void* x,
+                              const float* x_scale, int32_t* topk_idx, float* topk_w,
+                              int32_t* counts, int32_t* expert_off, void* recv, float* recv_scale,
+                              int32_t* slot_of, int32_t* src_of, void* ws, moe_stream_t stream) {
+  moe_status s = check_call(p, n, ws);
+  if (s != MOE_OK) return s;
+  if (!counts || !expert_off) return MOE_ERR_INVALID_ARG;
+  if (n > 0) {
+    if (!logits || !topk_idx || !topk_w || !x || !recv || !slot_of || !src_of)
+      return MOE_ERR_INVALID_ARG;
+    if (!aligned16(logits) || !aligned16(x) || !aligned16(recv)) return MOE_ERR_INVALID_ARG;
+    if (p->scale_cols > 0 && (!x_scale || !recv_scale)) return MOE_ERR_INVALID_ARG;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (route_blocks(n) <= kFusedMaxBlocks)
+    return cuda_status(launch_route_dispatch(*p, n, logits, x, x_scale, topk_idx, topk_w, counts,
+                                             expert_off, recv, recv_scale, slot_of, src_of, ws,
+                                             st));
+  s = cuda_status(launch_route(*p, n, logits, topk_idx, topk_w, counts, expert_off, ws, st));
+  if (s != MOE_OK) return s;
+  return cuda_status(launch_dispatch(*p, n, x, x_scale, topk_idx, recv, recv_scale, slot_of,
+                                     src_of, ws, st));
+}
+
 moe_status moe_expert_dequant(const moe_plan* p, int32_t n, const void* recv,
                               const float* recv_scale, const int32_t* slot_of, void* y, void* ws,
                               moe_stream_t stream) {
@@ -249,10 +273,9 @@ moe_status moe_layer(const moe_plan* p, int32_t n, const float* logits, const vo
   float* recv_scale = p->scale_cols > 0 ? reinterpret_cast<float*>(b + L.recv_scale) : nullptr;
   void* y = b + L.y;
   void* h = b + L.h;
-  s = moe_route_topk(p, n, logits, topk_idx, topk_w, counts, expert_off, ws, stream);
+  s = moe_route_dispatch(p, n, logits, x, x_scale, topk_idx, topk_w, counts, expert_off, recv,
+                         recv_scale, slot_of, src_of, ws, stream);
   if (s != MOE_OK || n == 0) return s;
-  s = moe_dispatch(p, n, x, x_scale, topk_idx, recv, recv_scale, slot_of, src_of, ws, stream);
-  if (s != MOE_OK) return s;
   const void* yin = recv;
   if (d.inter > 0) {
     s = moe_expert_swiglu(p, n, recv, counts, expert_off, w_gate_up, w_down, h, y, ws, stream);

@@ -17,6 +17,9 @@ constexpr int kRouteTokens = 32;
 constexpr int kRouteThreads = 1024;
 constexpr int kMaxExperts = 512;
 constexpr int kMaxTopK = 32;
+// Largest batch, in route blocks, that the fused route + dispatch launch
+// takes (n <= 1024 tokens); larger batches run the two kernels.
+constexpr int kFusedMaxBlocks = 32;
 
 // Control words at the start of every workspace.
 struct Ctrl {
@@ -76,6 +79,11 @@ cudaError_t launch_route_on(const moe_plan& p, int32_t n, const float* logits, i
 cudaError_t launch_dispatch(const moe_plan& p, int32_t n, const void* x, const float* x_scale,
                             const int32_t* topk_idx, void* recv, float* recv_scale,
                             int32_t* slot_of, int32_t* src_of, void* ws, cudaStream_t st);
+cudaError_t launch_route_dispatch(const moe_plan& p, int32_t n, const float* logits,
+                                  const void* x, const float* x_scale, int32_t* topk_idx,
+                                  float* topk_w, int32_t* counts, int32_t* expert_off, void* recv,
+                                  float* recv_scale, int32_t* slot_of, int32_t* src_of, void* ws,
+                                  cudaStream_t st);
 cudaError_t launch_dequant(const moe_plan& p, int32_t n, const void* recv, const float* recv_scale,
                            const int32_t* slot_of, void* y, void* ws, cudaStream_t st);
 cudaError_t launch_combine(const moe_plan& p, int32_t n, const void* y, const float* topk_w,

@@ -16,6 +16,7 @@
  *   moe_dispatch     copies every token row to its k expert slots
  *                    ("MLX expert parallelism all_to_all PR 3158", Facts:
  *                    dispatch_local / dispatch_scatter_remote).
+ *   moe_route_dispatch  the two calls above as one launch for small batches.
  *   moe_expert_*     the expert step reading the dispatched buffer in place:
  *                    grouped GEMMs read the rank-major buffer instead of a
  *                    per-expert copy (arXiv 2611.13188 abstract); segments are
@@ -147,6 +148,21 @@ MOE_API moe_status moe_route_topk(const moe_plan* plan, int32_t n, const float* 
 MOE_API moe_status moe_dispatch(const moe_plan* plan, int32_t n, const void* x, const float* x_scale,
                         const int32_t* topk_idx, void* recv, float* recv_scale,
                         int32_t* slot_of, int32_t* src_of, void* ws, moe_stream_t stream);
+
+/* Route and dispatch in one call: the results of moe_route_topk followed by
+ * moe_dispatch with the same arguments, bit for bit (same buffers, same
+ * layouts, same errors).  For n <= 1024 tokens both run in ONE cooperative
+ * launch with a single grid barrier: the decode-size step where fixed
+ * per-launch costs outweigh the bytes moved (the small-batch regime of "One-
+ * Sided Expert-Parallel All-to-All for Mixture-of-Experts Inference over
+ * NVLink", abstract).  Larger n runs the two kernels.  n = 0 writes zero
+ * counts and offsets only.  No counterpart call on the pages: it fuses two
+ * of their steps. */
+MOE_API moe_status moe_route_dispatch(const moe_plan* plan, int32_t n, const float* logits,
+                                      const void* x, const float* x_scale, int32_t* topk_idx,
+                                      float* topk_w, int32_t* counts, int32_t* expert_off,
+                                      void* recv, float* recv_scale, int32_t* slot_of,
+                                      int32_t* src_of, void* ws, moe_stream_t stream);
 
 /* Identity expert for FP8 rows: Y[s, c] = round_y(code[s, c] * recv_scale[s,
  * c / scale_block]) for every filled slot s = slot_of[t, j], correctly rounded

@@ -35,20 +35,28 @@ def numpy_inputs(inp: dict) -> dict:
     return {k: workloads.as_numpy_bits(v) for k, v in inp.items()}
 
 
-def run_gpu(cfg, inp: dict, plan=None, n_max=None, want=("all",)) -> dict:
-    """route -> dispatch -> (dequant) -> combine on cuda:0 via the C-ABI."""
+def run_gpu(cfg, inp: dict, plan=None, n_max=None, want=("all",), fused=False,
+            ws=None) -> dict:
+    """route -> dispatch -> (dequant) -> combine on cuda:0 via the C-ABI;
+    with fused=True route + dispatch go through moe_route_dispatch."""
     import combine_moe_route_11_b200 as mr
     n = inp["logits"].shape[0]
     dev = torch.device("cuda", 0)
     plan = plan or mr.Plan.from_config(cfg, n_max=n_max or max(n, 1))
-    ws = plan.new_workspace(dev)
+    ws = plan.new_workspace(dev) if ws is None else ws
     b = plan.new_buffers(n, dev)
     logits = inp["logits"].to(dev)
     x = inp["x"].to(dev)
     xs = inp["x_scale"].to(dev) if inp.get("x_scale") is not None else None
-    mr.moe_route_topk(plan, logits, b["topk_idx"], b["topk_w"], b["counts"], b["expert_off"], ws)
-    mr.moe_dispatch(plan, x, xs, b["topk_idx"], b["recv"], b["recv_scale"], b["slot_of"],
-                    b["src_of"], ws)
+    if fused:
+        mr.moe_route_dispatch(plan, logits, x, xs, b["topk_idx"], b["topk_w"], b["counts"],
+                              b["expert_off"], b["recv"], b["recv_scale"], b["slot_of"],
+                              b["src_of"], ws)
+    else:
+        mr.moe_route_topk(plan, logits, b["topk_idx"], b["topk_w"], b["counts"],
+                          b["expert_off"], ws)
+        mr.moe_dispatch(plan, x, xs, b["topk_idx"], b["recv"], b["recv_scale"], b["slot_of"],
+                        b["src_of"], ws)
     if cfg.x_dtype == "fp8_e4m3":
         mr.moe_expert_dequant(plan, n, b["recv"], b["recv_scale"], b["slot_of"], b["y"], ws)
         y = b["y"]

@@ -1,0 +1,108 @@
+"""moe_route_dispatch (one cooperative launch for n <= 1024 tokens) against the
+CPU oracle and against the two-call path, through the C ABI.
+
+The fused call must give exactly what moe_route_topk followed by moe_dispatch
+gives: every integer result and every dispatched byte bit-exact, gate weights
+within the same 8-ulp bound.  It shares the workspace's barrier generation and
+expert-total halves with the route kernel, so calls of both kinds are also
+interleaved on one workspace.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import parity
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+C = workloads.CONFIGS
+TINY = C["tiny"]
+
+# (name, config, n) -- every case runs the full oracle
+CASES = [
+    ("tiny", TINY, 64),
+    ("tiny_n1", TINY, 1),
+    ("tiny_n61", TINY, 61),
+    ("decode", C["decode"], 128),
+    ("decode_n33", C["decode"], 33),
+    ("prefill_fp8_ragged", C["prefill"], 300),
+    ("skewed_ragged", C["skewed"], 1000),
+    ("k1", TINY.replace(top_k=1), 100),
+    ("k_eq_E", TINY.replace(top_k=8, n_ranks=4), 70),
+    ("one_rank", TINY.replace(n_ranks=1), 90),
+    ("E6_scalar", TINY.replace(n_experts=6, top_k=3, n_ranks=3, hidden=64), 200),
+    ("E33_ragged_lanes", TINY.replace(n_experts=33, top_k=5, n_ranks=1, hidden=96), 150),
+    ("E512", TINY.replace(n_experts=512, top_k=8, n_ranks=8, hidden=128, x_dtype="bf16",
+                          y_dtype="bf16", out_dtype="bf16"), 130),
+    ("k16", TINY.replace(n_experts=32, top_k=16, n_ranks=2, hidden=64), 100),
+    # 32 route blocks: the largest batch the single launch takes
+    ("max_blocks_1024", TINY.replace(n_experts=64, top_k=6, n_ranks=4, hidden=32,
+                                     x_dtype="bf16", y_dtype="bf16", out_dtype="f32"), 1024),
+    # one token more: the call runs the two kernels
+    ("two_kernels_1025", TINY.replace(n_experts=64, top_k=6, n_ranks=4, hidden=32,
+                                      x_dtype="bf16", y_dtype="bf16", out_dtype="f32"), 1025),
+    ("fp8_small_D", C["prefill"].replace(hidden=256, n_experts=16, top_k=4, n_ranks=4), 129),
+]
+
+
+@pytest.mark.parametrize("name,cfg,n", CASES, ids=[c[0] for c in CASES])
+def test_fused_matches_oracle(name, cfg, n):
+    inp = workloads.make_inputs(cfg, seed=17, n=n)
+    inp_np = parity.numpy_inputs(inp)
+    ref = oracle.run_path(cfg, inp_np)
+    got = parity.run_gpu(cfg, inp, fused=True)
+    parity.compare_path(cfg, inp_np, ref, got)
+
+
+@pytest.mark.parametrize("name,n", [("decode", 128), ("prefill", 512), ("skewed", 1024)])
+def test_fused_equals_two_calls(name, n):
+    """Bit-exact agreement with moe_route_topk + moe_dispatch at workload
+    shapes, every output including the weights."""
+    cfg = C[name]
+    inp = workloads.make_inputs(cfg, seed=5, n=n)
+    a = parity.run_gpu(cfg, inp, fused=True)
+    b = parity.run_gpu(cfg, inp, fused=False)
+    assert a["status"] == 0 and b["status"] == 0
+    for key in ("topk_idx", "topk_w", "counts", "expert_off", "slot_of", "out"):
+        assert np.array_equal(a[key], b[key]), key
+    filled = np.sort(b["slot_of"].reshape(-1))
+    for key in ("src_of", "recv", "recv_scale", "y"):
+        if key in b:
+            assert np.array_equal(a[key][filled], b[key][filled]), key
+
+
+def test_fused_and_route_interleave_on_one_workspace():
+    """The two launch kinds alternate on one workspace.  The route kernel
+    keeps its expert totals in two halves chosen by the barrier generation;
+    the fused kernel also bumps the generation, so it must leave the half the
+    next route call uses at zero."""
+    import combine_moe_route_11_b200 as mr
+    cfg = TINY.replace(n_experts=16, top_k=4, n_ranks=4, hidden=64)
+    plan = mr.Plan.from_config(cfg, n_max=420)
+    ws = plan.new_workspace(torch.device("cuda", 0))
+    order = [False, True, False, True, False, False, True, True, False, True]
+    for i, fused in enumerate(order):
+        n = 37 + 41 * i
+        inp = workloads.make_inputs(cfg, seed=100 + i, n=n)
+        inp_np = parity.numpy_inputs(inp)
+        ref = oracle.run_path(cfg, inp_np)
+        got = parity.run_gpu(cfg, inp, plan=plan, fused=fused, ws=ws)
+        parity.compare_path(cfg, inp_np, ref, got)
+
+
+def test_fused_zero_tokens():
+    import combine_moe_route_11_b200 as mr
+    plan = mr.Plan.from_config(TINY, n_max=64)
+    dev = torch.device("cuda", 0)
+    ws = plan.new_workspace(dev)
+    b = plan.new_buffers(0, dev)
+    b["counts"].fill_(-7)
+    b["expert_off"].fill_(-7)
+    mr.moe_route_dispatch(plan, torch.empty(0, 8, device=dev), torch.empty(0, 256, device=dev),
+                          None, b["topk_idx"], b["topk_w"], b["counts"], b["expert_off"],
+                          b["recv"], None, b["slot_of"], b["src_of"], ws)
+    assert mr.moe_get_status(plan, ws) == 0
+    assert int(b["counts"].abs().sum()) == 0
+    assert int(b["expert_off"].abs().sum()) == 0
