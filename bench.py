@@ -63,6 +63,11 @@ def algorithmic_bytes(cfg, n: int) -> dict:
             "combine": combine, "step": route + dispatch + combine}
 
 
+# moe_route_dispatch runs route and dispatch as one launch up to this batch
+# (the library's documented limit; the binding carries the same constant)
+FUSED_MAX_TOKENS = 1024
+
+
 def describe(cfg, n: int) -> str:
     s = (f"{cfg.name}: N={n}, D={cfg.hidden}, E={cfg.n_experts}, k={cfg.top_k}, "
          f"R={cfg.n_ranks}, x={cfg.x_dtype}")
@@ -80,7 +85,9 @@ def step_config(cfg, n: int, n_sets: int, world: int, graph: bool = False) -> di
             "l2": (f"no flush: {n_sets} buffer set(s) rotate so a step's data was last touched "
                    f">= 4x L2 ({step_bytes * max(1, n_sets - 1) / 1e6:.0f} MB of traffic) "
                    f"earlier; steps run back to back"),
-            "timed": "route(top-k+counts+scan) + dispatch + combine, 3 launches/step",
+            "timed": ("moe_route_dispatch (route: top-k + counts + scan, then dispatch) + "
+                      "moe_combine: " + ("2 launches/step (route and dispatch fused)"
+                                         if n <= FUSED_MAX_TOKENS else "3 launches/step")),
             "y_source": "identity expert output, produced once before timing"}
 
 

@@ -21,7 +21,7 @@ OBJ_DIR = os.path.join(PKG, "_build")
 
 SOURCES = ["api.cu", "route.cu", "route_dispatch.cu", "dispatch.cu", "combine.cu", "swiglu_gemm.cu",
            "route_noalloc.cu"]
-HEADERS = ["moe_internal.cuh"]
+HEADERS = ["moe_internal.cuh", "route_common.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]

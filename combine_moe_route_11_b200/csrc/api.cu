@@ -54,7 +54,11 @@ Layout make_layout(const moe_plan& p) {
     return here;
   };
   L.ctrl = take(sizeof(Ctrl));
-  L.totals = take(size_t(2) * d.n_experts * 4);  // right after ctrl: cleared together
+  // right after ctrl, all cleared together by moe_workspace_init: expert totals
+  // [2, E] and token masks [2, mask rows, E], each double-buffered by the
+  // grid-barrier generation
+  L.totals = take(size_t(2) * d.n_experts * 4);
+  L.masks = take(size_t(2) * mask_rows(p) * d.n_experts * 4);
   L.blk = take(size_t(p.blocks_max) * d.n_experts * 4);
   L.bases = take(size_t(p.blocks_max) * d.n_experts * 4);
   L.rank = take(size_t(d.n_max) * d.top_k);
@@ -302,7 +306,7 @@ moe_status moe_get_status(const moe_plan* p, void* ws, moe_stream_t stream) {
 
 moe_status moe_workspace_init(const moe_plan* p, void* ws, moe_stream_t stream) {
   if (!p || !ws) return MOE_ERR_INVALID_ARG;
-  // control words and the expert totals (which follow them)
+  // control words, expert totals and token masks (which follow them)
   return cudaMemsetAsync(ws, 0, p->lay.blk, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
              ? MOE_OK
              : MOE_ERR_CUDA;

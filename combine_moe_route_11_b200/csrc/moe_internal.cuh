@@ -41,7 +41,7 @@ inline int elem_bytes(int dtype) {
 
 // Byte offsets of every buffer inside a workspace, fixed by n_max.
 struct Layout {
-  size_t ctrl, blk, bases, totals, rank, route_end;
+  size_t ctrl, totals, masks, blk, bases, rank, route_end;
   size_t topk_idx, topk_w, counts, expert_off, slot_of, src_of, recv, recv_scale, y, h, end;
 };
 
@@ -63,6 +63,10 @@ inline int64_t region_rows(const moe_plan& p, int32_t n) {
 }
 inline int64_t total_rows(const moe_plan& p, int32_t n) { return region_rows(p, n) * p.d.n_ranks; }
 inline int route_blocks(int32_t n) { return n <= 0 ? 1 : (n + kRouteTokens - 1) / kRouteTokens; }
+// Rows of each half of the fused kernel's [2, rows, E] token-mask table.
+inline int mask_rows(const moe_plan& p) {
+  return p.blocks_max < kFusedMaxBlocks ? p.blocks_max : kFusedMaxBlocks;
+}
 
 int num_sms();  // of the current device (cached per device)
 // Raise a kernel's dynamic shared-memory limit once per device.
@@ -72,10 +76,11 @@ cudaError_t set_smem_limit(const void* kernel, int bytes);
 cudaError_t launch_route(const moe_plan& p, int32_t n, const float* logits, int32_t* topk_idx,
                          float* topk_w, int32_t* counts, int32_t* expert_off, void* ws,
                          cudaStream_t st);
+// masks may be null when no fused call shares the scratch.
 cudaError_t launch_route_on(const moe_plan& p, int32_t n, const float* logits, int32_t* topk_idx,
                             float* topk_w, int32_t* counts, int32_t* expert_off, void* ctrl,
-                            int32_t* blk, int32_t* bases, int32_t* totals, uint8_t* rank,
-                            cudaStream_t st);
+                            int32_t* blk, int32_t* bases, int32_t* totals, uint32_t* masks,
+                            uint8_t* rank, cudaStream_t st);
 cudaError_t launch_dispatch(const moe_plan& p, int32_t n, const void* x, const float* x_scale,
                             const int32_t* topk_idx, void* recv, float* recv_scale,
                             int32_t* slot_of, int32_t* src_of, void* ws, cudaStream_t st);

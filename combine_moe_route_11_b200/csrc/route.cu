@@ -160,9 +160,13 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(RouteArgs a) {
     for (int u = blockIdx.x; u < E; u += gridDim.x) scan_column<1>(a, u, tot, s_warp, s_off);
   }
   if (blockIdx.x == 0) {
-    // the other half starts the next call at zero
+    // the other halves start the next call (of either route kernel) at zero
     int32_t* next = a.totals + size_t(s_parity ^ 1u) * E;
     for (int e = tid; e < E; e += kRouteThreads) next[e] = 0;
+    if (a.masks) {
+      uint32_t* m = a.masks + size_t(s_parity ^ 1u) * a.mask_rows * E;
+      for (int i = tid; i < a.mask_rows * E; i += kRouteThreads) m[i] = 0u;
+    }
     if (tid == 0) a.expert_off[E] = a.R * a.region_rows;
   }
   grid_dependents_launch();
@@ -214,6 +218,8 @@ cudaError_t launch_route(const moe_plan& p, int32_t n, const float* logits, int3
   a.blk = reinterpret_cast<int32_t*>(w + p.lay.blk);
   a.bases = reinterpret_cast<int32_t*>(w + p.lay.bases);
   a.totals = reinterpret_cast<int32_t*>(w + p.lay.totals);
+  a.masks = reinterpret_cast<uint32_t*>(w + p.lay.masks);
+  a.mask_rows = mask_rows(p);
   a.rank = reinterpret_cast<uint8_t*>(w + p.lay.rank);
   a.ws = ws;
   a.n = n;
@@ -237,8 +243,8 @@ namespace moe {
 // first call) and rank ([n, k] bytes).
 cudaError_t launch_route_on(const moe_plan& p, int32_t n, const float* logits, int32_t* topk_idx,
                             float* topk_w, int32_t* counts, int32_t* expert_off, void* ctrl,
-                            int32_t* blk, int32_t* bases, int32_t* totals, uint8_t* rank,
-                            cudaStream_t st) {
+                            int32_t* blk, int32_t* bases, int32_t* totals, uint32_t* masks,
+                            uint8_t* rank, cudaStream_t st) {
   RouteArgs a;
   a.logits = logits;
   a.topk_idx = topk_idx;
@@ -248,6 +254,8 @@ cudaError_t launch_route_on(const moe_plan& p, int32_t n, const float* logits, i
   a.blk = blk;
   a.bases = bases;
   a.totals = totals;
+  a.masks = masks;
+  a.mask_rows = mask_rows(p);
   a.rank = rank;
   a.ws = ctrl;
   a.n = n;

@@ -22,6 +22,8 @@ struct RouteArgs {
   int32_t* blk;    // [blocks, E] per-block counts
   int32_t* bases;  // [blocks, E] per-block absolute base slots
   int32_t* totals; // [2, E] expert totals, the half of this call chosen by barrier parity
+  uint32_t* masks; // [2, mask_rows, E] token masks of the fused kernel (null: none)
+  int32_t mask_rows;
   uint8_t* rank;   // [n, k]: rank of (t, j) among the block's tokens picking e
   void* ws;
   int32_t n, E, K, R;
@@ -54,16 +56,19 @@ __device__ __forceinline__ int expert_of(int q, int lane) {
   else return q * 32 + lane;
 }
 
-// Top-k and softmax of token t by the calling warp; returns lane j's pick.
-template <int VPL, int VEC>
-__device__ __forceinline__ int route_token(const RouteArgs& a, int64_t t, int lane) {
-  const int E = a.E, K = a.K;
-  const float* row = a.logits + t * E;
+// Top-k and softmax of one logit row by the calling warp: lane j < K gets
+// pick j and its weight; *nonfinite tells whether a pick had a non-finite
+// logit (fewer than K finite values in the row).  kStream loads the row as
+// read-once data; otherwise it stays cached for other blocks reading it too.
+template <int VPL, int VEC, bool kStream>
+__device__ __forceinline__ int route_row(const float* row, int E, int K, int lane, float* w,
+                                         bool* nonfinite) {
   uint32_t key[VPL];
   if constexpr (VEC == 4) {
 #pragma unroll
     for (int q4 = 0; q4 < VPL / 4; ++q4) {
-      const float4 v = __ldcs(reinterpret_cast<const float4*>(row + q4 * 128) + lane);
+      const float4* p = reinterpret_cast<const float4*>(row + q4 * 128) + lane;
+      const float4 v = kStream ? __ldcs(p) : __ldg(p);
       key[4 * q4 + 0] = order_key(v.x);
       key[4 * q4 + 1] = order_key(v.y);
       key[4 * q4 + 2] = order_key(v.z);
@@ -73,7 +78,7 @@ __device__ __forceinline__ int route_token(const RouteArgs& a, int64_t t, int la
 #pragma unroll
     for (int q = 0; q < VPL; ++q) {
       const int e = expert_of<VEC>(q, lane);
-      key[q] = e < E ? order_key(__ldcs(row + e)) : 0u;
+      key[q] = e < E ? order_key(kStream ? __ldcs(row + e) : __ldg(row + e)) : 0u;
     }
   }
   // This lane's best two untaken values (strict compares keep the lower id
@@ -128,12 +133,24 @@ __device__ __forceinline__ int route_token(const RouteArgs& a, int64_t t, int la
   float s = ex;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(kFull, s, off);
-  if (lane < K) {
-    a.topk_idx[t * K + lane] = my_i;
-    a.topk_w[t * K + lane] = ex / s;
-  }
-  if (__any_sync(kFull, lane < K && my_key == 1u) && lane == 0) set_status(a.ws, MOE_ERR_NONFINITE);
+  *w = ex / s;
+  *nonfinite = __any_sync(kFull, lane < K && my_key == 1u);
   return my_i;
+}
+
+// Top-k and softmax of token t by the calling warp, written to topk_idx and
+// topk_w; returns lane j's pick.
+template <int VPL, int VEC>
+__device__ __forceinline__ int route_token(const RouteArgs& a, int64_t t, int lane) {
+  float w;
+  bool nonfinite;
+  const int e = route_row<VPL, VEC, true>(a.logits + t * a.E, a.E, a.K, lane, &w, &nonfinite);
+  if (lane < a.K) {
+    a.topk_idx[t * a.K + lane] = e;
+    a.topk_w[t * a.K + lane] = w;
+  }
+  if (nonfinite && lane == 0) set_status(a.ws, MOE_ERR_NONFINITE);
+  return e;
 }
 
 // Calls f(VPL, VEC) -- as std::integral_constant values -- with the logits

@@ -2,22 +2,28 @@
 // offsets and the row scatter in ONE cooperative launch.
 //
 // At decode sizes the work of each step is a few megabytes, so the fixed cost
-// of separate launches and of the route kernel's second phase dominates
-// ("One-Sided Expert-Parallel All-to-All for Mixture-of-Experts Inference over
-// NVLink", abstract: fixed costs dominate at small batch; "backends/mlx:
-// runtime MoE expert-sort for decode", Summary: decode skips the sort because
-// of its overhead).  Here:
+// of separate launches and of long serial phases dominates ("One-Sided
+// Expert-Parallel All-to-All for Mixture-of-Experts Inference over NVLink",
+// abstract: fixed costs dominate at small batch; "backends/mlx: runtime MoE
+// expert-sort for decode", Summary: decode skips the sort because of its
+// overhead).  Block c owns tokens c, c + G, c + 2G, ... (G blocks), so the
+// routing of a batch is spread over as many SMs as it has tokens:
 //  1. every warp issues the load of its first 512-byte chunk of x (it does
-//     not depend on routing), then the blocks that own a route block of 32
-//     tokens route it exactly as the route kernel does (same per-token code):
-//     top-k, softmax, in-block ranks and the block's per-expert counts;
+//     not depend on routing); then one warp per owned token routes it (the
+//     same per-row code as the route kernel), keeps the picks in shared
+//     memory, writes topk_idx / topk_w, and sets the token's bit in the
+//     global mask of each picked expert for its 32-token route block
+//     (integer atomics: the resulting masks do not depend on their order);
 //  2. one bounded grid barrier;
-//  3. every block rebuilds the whole [blocks, E] base table in shared memory
-//     from the block counts (at most 32 route blocks, so a column is a few
-//     loads): expert totals, their exclusive prefix, the rank-major offsets
-//     and each block's base -- no second barrier;
-//  4. each warp stores its chunk to the token's k slots (base + rank), and
-//     the first chunk of a row carries the scales and the index maps.
+//  3. every block reads the [blocks, E] masks, and from their popcounts
+//     builds the expert totals, the exclusive prefix, the rank-major offsets
+//     and each route block's base slot, all in shared memory;
+//  4. the block's warps store the chunks of its tokens to their k slots:
+//     base + popcount of the lower tokens' bits in the mask, the same
+//     (expert, source token) order as the two-kernel path.
+// The mask table is double-buffered by the barrier generation: the half a
+// call uses was zeroed by the previous call of either route kernel, and each
+// call zeroes the other half for the next one.
 // Results are identical to moe_route_topk followed by moe_dispatch.
 #include "route_common.cuh"
 
@@ -36,61 +42,65 @@ struct FusedArgs {
   int32_t vecs;     // 16-byte vectors per row
   int32_t chunks;   // 512-byte chunks per row
   int32_t total;    // T
+  int32_t owned;    // most tokens any block owns: ceil(n / grid)
 };
 
 template <int VPL, int VEC>
 __global__ void __launch_bounds__(kRouteThreads, 1) route_dispatch_kernel(FusedArgs f) {
-  extern __shared__ int32_t s_base[];                 // [blocks, E] absolute bases
-  __shared__ int32_t s_sel[kRouteTokens * kMaxTopK];  // picks of the block's tokens
-  __shared__ uint32_t s_mask[kMaxExperts];            // token mask per expert
-  __shared__ int32_t s_pre[kMaxExperts];              // exclusive prefix of expert totals
+  extern __shared__ int32_t s_dyn[];  // masks [blocks, E], bases [blocks, E], picks [owned, K]
+  __shared__ int32_t s_pre[kMaxExperts];
   __shared__ int32_t s_wsum[kWarps];
   __shared__ unsigned s_parity;
   const RouteArgs& a = f.r;
-  const int E = a.E, K = a.K, B = a.blocks;
+  const int E = a.E, K = a.K, B = a.blocks, n = a.n;
+  const int G = gridDim.x;
+  uint32_t* s_mask = reinterpret_cast<uint32_t*>(s_dyn);
+  int32_t* s_base = s_dyn + B * E;
+  int32_t* s_pick = s_dyn + 2 * B * E;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t row_bytes = int64_t(f.vecs) << 4;
-  const int64_t n_items = int64_t(a.n) * f.chunks;
-  const int64_t first = int64_t(blockIdx.x) * kWarps + warp;
-  const int64_t stride = int64_t(gridDim.x) * kWarps;
+  // tokens of this block: blockIdx.x + i * G for i < mine
+  const int mine = int(blockIdx.x) < n ? (n - 1 - int(blockIdx.x)) / G + 1 : 0;
+  const int items = mine * f.chunks;  // (owned token i, chunk c) -> i * chunks + c
   grid_dependency_wait();
+  if (tid == 0) s_parity = ld_acquire_gpu(&reinterpret_cast<Ctrl*>(a.ws)->gen) & 1u;
 
   // ---- the first chunk of x, in flight while routing runs
   uint4 v0 = make_uint4(0u, 0u, 0u, 0u);
-  if (first < n_items) {
-    const int64_t t = first / f.chunks;
-    const int64_t g = int64_t(first % f.chunks) * 32 + lane;
+  if (warp < items) {
+    const int64_t t = blockIdx.x + int64_t(warp / f.chunks) * G;
+    const int64_t g = int64_t(warp % f.chunks) * 32 + lane;
     if (g < f.vecs) v0 = ld_nc_v4(f.x + t * row_bytes + (g << 4));
   }
-  if (blockIdx.x == 0 && tid == 0) s_parity = ld_acquire_gpu(&reinterpret_cast<Ctrl*>(a.ws)->gen) & 1u;
+  __syncthreads();
+  uint32_t* gmask = a.masks + size_t(s_parity) * a.mask_rows * E;
 
-  // ---- phase 1: route blocks b = blockIdx.x, blockIdx.x + grid, ...
-  for (int b = blockIdx.x; b < B; b += gridDim.x) {
-    const int t_base = b * kRouteTokens;
-    const int valid = max(0, min(kRouteTokens, a.n - t_base));
-    for (int i = tid; i < E; i += kRouteThreads) s_mask[i] = 0;
-    if (warp < valid) {
-      const int e = route_token<VPL, VEC>(a, int64_t(t_base) + warp, lane);
-      if (lane < K) s_sel[warp * K + lane] = e;
+  // ---- phase 1: one warp per owned token
+  for (int i = warp; i < mine; i += kWarps) {
+    const int t = int(blockIdx.x) + i * G;
+    float w;
+    bool nonfinite;
+    const int e = route_row<VPL, VEC, true>(a.logits + int64_t(t) * E, E, K, lane, &w, &nonfinite);
+    if (lane < K) {
+      s_pick[i * K + lane] = e;
+      a.topk_idx[int64_t(t) * K + lane] = e;
+      a.topk_w[int64_t(t) * K + lane] = w;
+      atomicOr(&gmask[(t / kRouteTokens) * E + e], 1u << (t % kRouteTokens));
     }
-    __syncthreads();
-    for (int p = tid; p < valid * K; p += kRouteThreads)
-      atomicOr(&s_mask[s_sel[p]], 1u << (p / K));
-    __syncthreads();
-    for (int p = tid; p < valid * K; p += kRouteThreads) {
-      const int tl = p / K;
-      a.rank[int64_t(t_base) * K + p] = uint8_t(__popc(s_mask[s_sel[p]] & ((1u << tl) - 1u)));
-    }
-    for (int e = tid; e < E; e += kRouteThreads) a.blk[int64_t(b) * E + e] = __popc(s_mask[e]);
-    __syncthreads();
+    if (nonfinite && lane == 0) set_status(a.ws, MOE_ERR_NONFINITE);
   }
 
-  if (!grid_barrier(a.ws, gridDim.x)) return;
+  if (!grid_barrier(a.ws, G)) return;
 
-  // ---- phase 2, in every block: expert totals, offsets and the base table
+  // ---- phase 2, in every block: masks, totals, offsets and the base table
   int tot = 0;
-  if (tid < E)
-    for (int b = 0; b < B; ++b) tot += __ldcg(a.blk + int64_t(b) * E + tid);
+  if (tid < E) {
+    for (int b = 0; b < B; ++b) {
+      const uint32_t m = __ldcg(gmask + b * E + tid);
+      s_mask[b * E + tid] = m;
+      tot += __popc(m);
+    }
+  }
   int incl = tot;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -120,7 +130,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_dispatch_kernel(FusedA
     int run = off;
     for (int b = 0; b < B; ++b) {
       s_base[b * E + tid] = run;
-      run += __ldcg(a.blk + int64_t(b) * E + tid);
+      run += __popc(s_mask[b * E + tid]);
     }
     if (blockIdx.x == 0) {
       a.counts[tid] = tot;
@@ -129,26 +139,31 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_dispatch_kernel(FusedA
       a.totals[size_t(s_parity ^ 1u) * E + tid] = 0;
     }
   }
-  if (blockIdx.x == 0 && tid == 0) a.expert_off[E] = a.R * a.region_rows;
+  if (blockIdx.x == 0) {
+    uint32_t* next = a.masks + size_t(s_parity ^ 1u) * a.mask_rows * E;
+    for (int i = tid; i < a.mask_rows * E; i += kRouteThreads) next[i] = 0u;
+    if (tid == 0) a.expert_off[E] = a.R * a.region_rows;
+  }
   __syncthreads();
 
-  // ---- phase 3: each warp's chunks to the k slots of their token
-  for (int64_t item = first; item < n_items; item += stride) {
-    const int64_t t = item / f.chunks;
-    const int c = int(item % f.chunks);
+  // ---- phase 3: the chunks of this block's tokens to their k slots
+  for (int it = warp; it < items; it += kWarps) {
+    const int i = it / f.chunks, c = it % f.chunks;
+    const int t = int(blockIdx.x) + i * G;
     const int64_t g = int64_t(c) * 32 + lane;
     uint4 v = v0;
-    if (item != first && g < f.vecs) v = ld_nc_v4(f.x + t * row_bytes + (g << 4));
+    if (it != warp && g < f.vecs) v = ld_nc_v4(f.x + int64_t(t) * row_bytes + (g << 4));
     int slot = -1;
     if (lane < K) {
-      const int64_t tk = t * K + lane;
-      const int e = __ldcg(a.topk_idx + tk);
+      const int e = s_pick[i * K + lane];
       if (e >= 0 && e < E) {
-        slot = s_base[int(t / kRouteTokens) * E + e] + __ldcg(a.rank + tk);
+        const int b = t / kRouteTokens, tl = t % kRouteTokens;
+        slot = s_base[b * E + e] + __popc(s_mask[b * E + e] & ((1u << tl) - 1u));
         if (slot < 0 || slot >= f.total) slot = -1;
       }
       if (slot < 0) set_status(a.ws, MOE_ERR_DEVICE_INDEX);
       if (c == 0) {
+        const int64_t tk = int64_t(t) * K + lane;
         f.slot_of[tk] = slot;
         if (slot >= 0) f.src_of[slot] = int32_t(tk);
       }
@@ -160,11 +175,11 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_dispatch_kernel(FusedA
     }
     if (c == 0 && f.S > 0) {
       for (int i0 = 0; i0 < f.S; i0 += 32) {
-        const int i = i0 + lane;
-        const float sv = i < f.S ? __ldcs(f.x_scale + t * f.S + i) : 0.f;
+        const int si = i0 + lane;
+        const float sv = si < f.S ? __ldcs(f.x_scale + int64_t(t) * f.S + si) : 0.f;
         for (int j = 0; j < K; ++j) {
           const int s = __shfl_sync(kFull, slot, j);
-          if (s >= 0 && i < f.S) __stcs(f.recv_scale + int64_t(s) * f.S + i, sv);
+          if (s >= 0 && si < f.S) __stcs(f.recv_scale + int64_t(s) * f.S + si, sv);
         }
       }
     }
@@ -172,10 +187,19 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_dispatch_kernel(FusedA
   grid_dependents_launch();
 }
 
+// Dynamic shared memory of a launch: masks and bases [blocks, E] and the
+// owned tokens' picks [owned, K].
+size_t fused_smem(int blocks, int E, int owned, int K) {
+  return (2 * size_t(blocks) * E + size_t(owned) * K) * 4;
+}
+
 template <int VPL, int VEC>
-cudaError_t launch_fused(const FusedArgs& f, int sms, cudaStream_t st) {
+cudaError_t launch_fused(FusedArgs f, int sms, cudaStream_t st) {
   static int per_sm[64] = {0};  // resident blocks per SM, per device
-  constexpr int kMaxDyn = kFusedMaxBlocks * kMaxExperts * 4;
+  // largest use: 32 route blocks of 512 experts, and the picks of up to 64
+  // owned tokens of top-k 32 (1024 tokens need a grid of at least 16 blocks)
+  constexpr int kMaxOwned = 64;
+  const int kMaxDyn = int(fused_smem(kFusedMaxBlocks, kMaxExperts, kMaxOwned, kMaxTopK));
   auto kernel = route_dispatch_kernel<VPL, VEC>;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -190,14 +214,15 @@ cudaError_t launch_fused(const FusedArgs& f, int sms, cudaStream_t st) {
     if (nb < 1) return cudaErrorInvalidConfiguration;
     per_sm[dev] = nb;
   }
-  const int64_t items = int64_t(f.r.n) * f.chunks;
-  int64_t grid = (items + kWarps - 1) / kWarps;
-  if (grid < f.r.blocks) grid = f.r.blocks;
+  // one block per token up to the resident limit
+  int64_t grid = f.r.n > 1 ? f.r.n : 1;
   if (grid > int64_t(per_sm[dev]) * sms) grid = int64_t(per_sm[dev]) * sms;
+  f.owned = int32_t((int64_t(f.r.n) + grid - 1) / grid);
+  if (f.owned > kMaxOwned) return cudaErrorNotSupported;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned(grid));
   cfg.blockDim = dim3(kRouteThreads);
-  cfg.dynamicSmemBytes = size_t(f.r.blocks) * f.r.E * 4;
+  cfg.dynamicSmemBytes = fused_smem(f.r.blocks, f.r.E, f.owned, f.r.K);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;
@@ -225,6 +250,8 @@ cudaError_t launch_route_dispatch(const moe_plan& p, int32_t n, const float* log
   a.blk = reinterpret_cast<int32_t*>(w + p.lay.blk);
   a.bases = reinterpret_cast<int32_t*>(w + p.lay.bases);
   a.totals = reinterpret_cast<int32_t*>(w + p.lay.totals);
+  a.masks = reinterpret_cast<uint32_t*>(w + p.lay.masks);
+  a.mask_rows = mask_rows(p);
   a.rank = reinterpret_cast<uint8_t*>(w + p.lay.rank);
   a.ws = ws;
   a.n = n;
@@ -243,7 +270,8 @@ cudaError_t launch_route_dispatch(const moe_plan& p, int32_t n, const float* log
   f.vecs = int32_t(int64_t(p.d.hidden) * elem_bytes(p.d.x_dtype) / 16);
   f.chunks = (f.vecs + 31) / 32;
   f.total = int32_t(total_rows(p, n));
-  if (a.blocks > kFusedMaxBlocks) return cudaErrorInvalidValue;
+  f.owned = 0;
+  if (a.blocks > a.mask_rows) return cudaErrorInvalidValue;
   const int sms = num_sms();
   return with_route_shape(a.E, [&](auto vpl, auto vec) {
     return launch_fused<decltype(vpl)::value, decltype(vec)::value>(f, sms, st);

@@ -69,7 +69,7 @@ extern "C" MOE_API moe_status moe_route_topk_noalloc(const moe_plan* p, int32_t 
   if (cudaMemsetAsync(b, 0, sizeof(moe::Ctrl) + totals_bytes, st) != cudaSuccess)
     return MOE_ERR_CUDA;
   const cudaError_t e = moe::launch_route_on(*p, n, logits, topk_idx, topk_w, counts, expert_off,
-                                             b, blk, bases, totals, rank, st);
+                                             b, blk, bases, totals, nullptr, rank, st);
   if (e == cudaSuccess) return MOE_OK;
   return e == cudaErrorNotSupported ? MOE_ERR_UNSUPPORTED : MOE_ERR_CUDA;
 }

@@ -21,8 +21,14 @@
 //               or conversion (GEMM2), bf16 stores of the valid rows.
 // Tiles (expert, n-tile, m-tile) are enumerated on the device from the
 // routing counts, m-tile innermost so the CTAs sharing a weight tile run at
-// the same time.  Rows of a tile past the expert's segment are computed and
-// not stored.  Every wait is bounded; on timeout the CTA records
+// the same time.  An expert's last m-tile usually holds only a few rows;
+// when it holds at most 96, the tile swaps the operand roles -- the weight
+// rows become the MMA's M side (two M=128 halves) and the token rows its N
+// side, rounded up to 16 -- so the tensor cores do work in proportion to
+// the rows present instead of a full 128.  Its accumulators are transposed
+// (TMEM lane = weight row, column = token) and the epilogue stores them
+// transposed.  Rows of a normal tile past the expert's segment are computed
+// and not stored.  Every wait is bounded; on timeout the CTA records
 // MOE_ERR_TIMEOUT, drains its own copies and MMAs, frees its tensor memory
 // and returns.
 #include "moe_internal.cuh"
@@ -45,6 +51,7 @@ constexpr uint32_t kABytes = kBM * kBK * 2;
 constexpr uint32_t kBBytes = kBN * kBK * 2;
 constexpr uint32_t kStageBytes = kABytes + kBBytes;
 constexpr int kMaxE = kMaxExperts;
+constexpr int kSwapMaxRows = 96;     // last m-tiles with at most this many rows swap roles
 constexpr size_t kSmemBytes = size_t(kStages) * kStageBytes + 1024 /*align*/ + 1024 /*meta*/;
 
 struct GemmArgs {
@@ -69,17 +76,19 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
          (uint64_t(1) << 46) | (uint64_t(2) << 61);
 }
 
-// kind::f16 instruction descriptor: bf16 A and B (K-major), fp32 D, M=128, N=256.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kBN >> 3) << 17) |
-                            (uint32_t(kBM >> 4) << 24);
+// kind::f16 instruction descriptor: bf16 A and B (K-major), fp32 D, M=128,
+// N = n (a multiple of 16, at most 256).
+__host__ __device__ constexpr uint32_t idesc_m128(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(n >> 3) << 17) | (uint32_t(kBM >> 4) << 24);
+}
 
 __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                          uint32_t accumulate) {
+                                          uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
+      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -127,6 +136,12 @@ struct Tile {
   int e, n, m;
 };
 
+// Rows of tile tl that belong to its expert (1..128), from the clamped counts.
+__device__ __forceinline__ int tile_rows(const Tile& tl, const int* s_cnt) {
+  return min(s_cnt[tl.e] - tl.m * kBM, kBM);
+}
+__device__ __forceinline__ bool swapped_tile(int rows) { return rows <= kSwapMaxRows; }
+
 // Tile t of the (expert, n-tile, m-tile) order with m innermost; s_pref[e] is
 // the number of m-tiles of the experts below e.
 __device__ __forceinline__ Tile tile_of(int t, const int* s_pref, int E, int n_tiles) {
@@ -163,6 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drained + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
   __shared__ int s_pref[kMaxE + 1];
+  __shared__ int s_cnt[kMaxE];  // counts clamped to [0, T]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = g.E;
@@ -193,7 +209,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     int carry = 0;
     for (int e0 = 0; e0 < E; e0 += 32) {
       const int e = e0 + lane;
-      const int mt = e < E ? (min(max(g.counts[e], 0), g.total) + kBM - 1) / kBM : 0;
+      const int c = e < E ? min(max(g.counts[e], 0), g.total) : 0;
+      if (e < E) s_cnt[e] = c;
+      const int mt = (c + kBM - 1) / kBM;
       int incl = mt;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -261,6 +279,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + uint32_t(acc * kBN);
+        const Tile tl = tile_of(t, s_pref, E, g.n_tiles);
+        const int rows = tile_rows(tl, s_cnt);
+        const bool swap = swapped_tile(rows);
+        // swapped: M = 128 weight rows per half, N = the tile's rows rounded up to 16
+        const uint32_t idesc = swap ? idesc_m128((rows + 15) & ~15) : idesc_m128(kBN);
         bool ok = true;
         for (int kb = 0; kb < g.k_steps; ++kb) {
           if (!mbar_wait(&full[stage], phase)) {
@@ -272,10 +295,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t a_addr = smem_addr(smem + size_t(stage) * kStageBytes);
           const uint32_t b_addr = a_addr + kABytes;
+          if (swap) {
 #pragma unroll
-          for (int k = 0; k < kBK / kUmmaK; ++k)
-            umma_bf16(d_tmem, smem_desc_sw128(a_addr + k * kUmmaK * 2),
-                      smem_desc_sw128(b_addr + k * kUmmaK * 2), (kb | k) != 0 ? 1u : 0u);
+            for (int k = 0; k < kBK / kUmmaK; ++k)
+#pragma unroll
+              for (int half = 0; half < 2; ++half)
+                umma_bf16(d_tmem + uint32_t(half * (kBN / 2)),
+                          smem_desc_sw128(b_addr + half * (kBBytes / 2) + k * kUmmaK * 2),
+                          smem_desc_sw128(a_addr + k * kUmmaK * 2), idesc,
+                          (kb | k) != 0 ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int k = 0; k < kBK / kUmmaK; ++k)
+              umma_bf16(d_tmem, smem_desc_sw128(a_addr + k * kUmmaK * 2),
+                        smem_desc_sw128(b_addr + k * kUmmaK * 2), idesc, (kb | k) != 0 ? 1u : 0u);
+          }
           umma_commit(&empty[stage]);  // stage free once these MMAs have read it
           if (++stage == kStages) stage = 0, phase ^= 1u;
         }
@@ -304,13 +338,55 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const int rows = min(g.counts[tl.e], g.total) - tl.m * kBM;
-      const int64_t row = int64_t(g.expert_off[tl.e]) + tl.m * kBM + r_local;
+      const int rows = tile_rows(tl, s_cnt);
+      const int64_t row0 = int64_t(g.expert_off[tl.e]) + tl.m * kBM;
+      const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(acc * kBN);
+      if (swapped_tile(rows)) {
+        // transposed accumulators: this thread's TMEM lane is weight row
+        // r_local of each half, column c is the tile's row c
+#pragma unroll 1
+        for (int c0 = 0; c0 < rows; c0 += 32) {
+          if (kSwiGLU) {
+            float gate[32], up[32];
+            tmem_ld32(taddr + uint32_t(c0), gate);
+            tmem_ld32(taddr + uint32_t(kBN / 2 + c0), up);
+            const int64_t f = int64_t(tl.n) * (kBN / 2) + r_local;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int64_t row = row0 + c0 + i;
+              if (c0 + i >= rows) break;
+              if (row < 0 || row >= g.total) {
+                set_status(g.ws, MOE_ERR_DEVICE_INDEX);
+                continue;
+              }
+              const float h = gate[i] / (1.f + expf(-gate[i])) * up[i];
+              g.out[row * g.out_ld + f] = __float2bfloat16_rn(h);
+            }
+          } else {
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+              float v[32];
+              tmem_ld32(taddr + uint32_t(half * (kBN / 2) + c0), v);
+              const int64_t f = int64_t(tl.n) * kBN + half * (kBN / 2) + r_local;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const int64_t row = row0 + c0 + i;
+                if (c0 + i >= rows) break;
+                if (row < 0 || row >= g.total) {
+                  set_status(g.ws, MOE_ERR_DEVICE_INDEX);
+                  continue;
+                }
+                g.out[row * g.out_ld + f] = __float2bfloat16_rn(v[i]);
+              }
+            }
+          }
+        }
+      } else {
+      const int64_t row = row0 + r_local;
       // a segment outside [0, T) (caller-supplied counts or offsets) is skipped
       const bool in_range = row >= 0 && row < g.total;
       const bool valid = r_local < rows && in_range;
       if (r_local < rows && !in_range) set_status(g.ws, MOE_ERR_DEVICE_INDEX);
-      const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(acc * kBN);
       if (kSwiGLU) {
         __nv_bfloat16* dst = g.out + row * g.out_ld + int64_t(tl.n) * (kBN / 2);
 #pragma unroll 1
@@ -348,6 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               d4[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
           }
         }
+      }
       }
       tc_fence_before();
       __syncwarp();

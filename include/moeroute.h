@@ -151,13 +151,15 @@ MOE_API moe_status moe_dispatch(const moe_plan* plan, int32_t n, const void* x, 
 
 /* Route and dispatch in one call: the results of moe_route_topk followed by
  * moe_dispatch with the same arguments, bit for bit (same buffers, same
- * layouts, same errors).  For n <= 1024 tokens both run in ONE cooperative
- * launch with a single grid barrier: the decode-size step where fixed
- * per-launch costs outweigh the bytes moved (the small-batch regime of "One-
- * Sided Expert-Parallel All-to-All for Mixture-of-Experts Inference over
- * NVLink", abstract).  Larger n runs the two kernels.  n = 0 writes zero
- * counts and offsets only.  No counterpart call on the pages: it fuses two
- * of their steps. */
+ * layouts, same errors).  For n <= 1024 tokens both run in ONE launch: the
+ * decode-size step where fixed per-launch costs outweigh the bytes moved (the
+ * small-batch regime of "One-Sided Expert-Parallel All-to-All for Mixture-of-
+ * Experts Inference over NVLink", abstract): a cooperative launch in which
+ * each block routes and scatters its own tokens, with a single grid barrier
+ * between routing and scattering.  Larger n runs the two kernels.  Unlike
+ * moe_route_topk, the one-launch form leaves no per-block bases in ws for a
+ * later moe_dispatch.  n = 0 writes zero counts and offsets only.  No
+ * counterpart call on the pages: it fuses two of their steps. */
 MOE_API moe_status moe_route_dispatch(const moe_plan* plan, int32_t n, const float* logits,
                                       const void* x, const float* x_scale, int32_t* topk_idx,
                                       float* topk_w, int32_t* counts, int32_t* expert_off,
@@ -215,9 +217,9 @@ MOE_API void* moe_layer_buffer(const moe_plan* plan, void* ws, const char* name)
  * (MOE_ERR_CUDA if the copy itself fails). */
 MOE_API moe_status moe_get_status(const moe_plan* plan, void* ws, moe_stream_t stream);
 
-/* Zero the control words and expert totals of a workspace (an alternative
- * to zero-filling it), enqueued on `stream`.  Required again after a call
- * reported MOE_ERR_TIMEOUT. */
+/* Zero the control words, expert totals and token masks of a workspace (an
+ * alternative to zero-filling it), enqueued on `stream`.  Required again
+ * after a call reported MOE_ERR_TIMEOUT. */
 MOE_API moe_status moe_workspace_init(const moe_plan* plan, void* ws, moe_stream_t stream);
 
 /* Bytes of the fixed scratch array that moe_route_topk_noalloc uses. */

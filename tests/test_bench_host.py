@@ -65,3 +65,15 @@ def test_algorithmic_bytes_and_rotation():
     nd = bench.buffer_sets(workloads.CONFIGS["decode"], 128)
     step = bench.algorithmic_bytes(workloads.CONFIGS["decode"], 128)["step"]
     assert (nd - 1) * step >= 4 * bench.L2_BYTES
+
+
+def test_fused_batch_limit_agrees_with_the_library():
+    """bench.py describes the step without importing the library (the
+    reference arm runs without it); its copy of the one-launch limit must be
+    the binding's, which the header documents (32 route blocks of 32)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import combine_moe_route_11_b200 as mr
+    assert bench.FUSED_MAX_TOKENS == mr.FUSED_MAX_TOKENS == 32 * 32
+    with open(os.path.join(ROOT, "include", "moeroute.h")) as f:
+        assert "n <= 1024 tokens" in f.read()

@@ -1,5 +1,6 @@
-"""moe_route_dispatch (one cooperative launch for n <= 1024 tokens) against the
-CPU oracle and against the two-call path, through the C ABI.
+"""moe_route_dispatch (one cooperative launch for n <= 1024 tokens, each block
+routing and scattering its own tokens around one grid barrier) against the CPU
+oracle and against the two-call path, through the C ABI.
 
 The fused call must give exactly what moe_route_topk followed by moe_dispatch
 gives: every integer result and every dispatched byte bit-exact, gate weights
@@ -37,6 +38,11 @@ CASES = [
     ("E512", TINY.replace(n_experts=512, top_k=8, n_ranks=8, hidden=128, x_dtype="bf16",
                           y_dtype="bf16", out_dtype="bf16"), 130),
     ("k16", TINY.replace(n_experts=32, top_k=16, n_ranks=2, hidden=64), 100),
+    ("E512_n128", TINY.replace(n_experts=512, top_k=8, n_ranks=8, hidden=128, x_dtype="bf16",
+                               y_dtype="bf16", out_dtype="bf16"), 128),
+    # more tokens than resident blocks: blocks own several tokens
+    ("owned_many_777", C["decode"].replace(hidden=512), 777),
+    ("decode_n257", C["decode"].replace(hidden=512), 257),
     # 32 route blocks: the largest batch the single launch takes
     ("max_blocks_1024", TINY.replace(n_experts=64, top_k=6, n_ranks=4, hidden=32,
                                      x_dtype="bf16", y_dtype="bf16", out_dtype="f32"), 1024),
@@ -74,10 +80,10 @@ def test_fused_equals_two_calls(name, n):
 
 
 def test_fused_and_route_interleave_on_one_workspace():
-    """The two launch kinds alternate on one workspace.  The route kernel
-    keeps its expert totals in two halves chosen by the barrier generation;
-    the fused kernel also bumps the generation, so it must leave the half the
-    next route call uses at zero."""
+    """The two launch kinds alternate on one workspace.  Both keep tables in
+    two halves chosen by the barrier generation (the route kernel's expert
+    totals, the fused kernel's token masks), and each must leave the halves
+    the next call of either kind uses at zero."""
     import combine_moe_route_11_b200 as mr
     cfg = TINY.replace(n_experts=16, top_k=4, n_ranks=4, hidden=64)
     plan = mr.Plan.from_config(cfg, n_max=420)

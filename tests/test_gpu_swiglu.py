@@ -63,12 +63,15 @@ def test_swiglu_small_matches_oracle(name, cfg, n):
     parity.assert_layer_out_close(parity.to_bits(b["out"]), ref)
 
 
-def test_swiglu_layer_shape_sampled_rows():
+@pytest.mark.parametrize("n,k", [(300, 4), (1000, 8)])
+def test_swiglu_layer_shape_sampled_rows(n, k):
     """Full D = 7168 and I = 2048 (E = 16 experts to bound the weight bytes):
     every output row of the GPU is checked on a sample of filled slots,
-    including the first and last row of every expert segment."""
-    cfg = LAYER.replace(n_experts=16, top_k=4, n_ranks=4)
-    n = 300
+    including the first and last row of every expert segment and the rows
+    on each side of every 128-row tile boundary.  At n=300, k=4 every expert
+    is one short tile (operand roles swapped); at n=1000, k=8 experts span
+    several full tiles and a last one."""
+    cfg = LAYER.replace(n_experts=16, top_k=k, n_ranks=4)
     inp = workloads.make_inputs(cfg, seed=7, n=n)
     _, _, b = run_layer_gpu(cfg, inp, n)
     off = b["expert_off"].cpu().numpy()
@@ -78,6 +81,8 @@ def test_swiglu_layer_shape_sampled_rows():
     for e in range(cfg.n_experts):
         if cnt[e]:
             slots += [off[e], off[e] + cnt[e] - 1, off[e] + cnt[e] // 2]
+            for edge in range(128, int(cnt[e]), 128):
+                slots += [off[e] + edge - 1, off[e] + edge]
     slots = np.unique(np.array(slots, np.int64))
     tok = src[slots] // cfg.top_k
     expert = np.searchsorted(off[:cfg.n_experts], slots, side="right") - 1
@@ -102,3 +107,32 @@ def test_layer_entry_point_with_swiglu():
                  inp["w_down"].to(dev), out, ws)
     assert mr.moe_get_status(plan, ws) == 0
     parity.assert_layer_out_close(parity.to_bits(out), ref)
+
+
+def test_swiglu_tile_shapes_from_designed_counts():
+    """Expert segments of 1, 16, 17, 96, 97, 128, 261 and 0 rows (k = 1, each
+    token sent to a chosen expert): last m-tiles of every size class -- swapped
+    roles with N = 16, 32 and 96, the first normal size (97), a full tile, a
+    full tile followed by a swapped tail, and an empty expert."""
+    counts = [1, 16, 17, 96, 97, 128, 261, 0]
+    cfg = LAYER.replace(hidden=512, inter=256, n_experts=8, top_k=1, n_ranks=2)
+    n = sum(counts)
+    inp = workloads.make_inputs(cfg, seed=13, n=n)
+    g = torch.Generator().manual_seed(14)
+    assign = torch.repeat_interleave(torch.arange(8), torch.tensor(counts))
+    assign = assign[torch.randperm(n, generator=g)]
+    logits = 0.1 * torch.randn(n, 8, generator=g)
+    logits[torch.arange(n), assign] = 10.0
+    inp["logits"] = logits
+    inp_np = parity.numpy_inputs(inp)
+    ref = oracle.run_path(cfg, inp_np)
+    assert list(ref["counts"]) == counts
+    _, _, b = run_layer_gpu(cfg, inp, n)
+    assert np.array_equal(parity.to_bits(b["slot_of"]), ref["slot_of"])
+    fs = np.sort(ref["slot_of"].reshape(-1))
+    expert_of_slot = ref["topk_idx"].reshape(-1)[ref["src_of"][fs]]
+    _, h_ref = oracle.swiglu_rows(fs, expert_of_slot, ref["recv"], inp_np["w_gate_up"],
+                                  inp_np["w_down"], want_h=True)
+    parity.assert_gemm_rows_close(parity.to_bits(b["h"])[fs], h_ref[fs], "H")
+    parity.assert_gemm_rows_close(parity.to_bits(b["y"])[fs], ref["y"][fs], "Y")
+    parity.assert_layer_out_close(parity.to_bits(b["out"]), ref)
