@@ -5,8 +5,10 @@
 // Inference over NVLink", abstract).  With R virtual ranks on one GPU, a
 // "remote" region is a byte range of the same HBM, so the push is a store.
 //
-// Work item = (token, 2 KB column chunk of its row), one warp each.  Every
-// lane loads 4 sixteen-byte vectors of the chunk first (they do not depend on
+// Work item = (token, 1 KB column chunk of its row), one warp each; 1 KB
+// divides both the 7168-byte FP8 rows and the 14336-byte bf16 rows of the
+// workloads, and 32 registers per thread let 8 blocks share an SM.  Every
+// lane loads 2 sixteen-byte vectors of the chunk first (they do not depend on
 // routing), while lanes j < k resolve the slot of choice j -- the route
 // call's per-block base plus the in-block rank, no metadata round trip --
 // then the warp stores the chunk k times.  Scales and the index maps go with
@@ -21,8 +23,8 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kVec = 4;                 // 16-byte vectors per lane per chunk
-constexpr int kChunkVec = 32 * kVec;    // vectors per chunk (2 KB)
+constexpr int kVec = 2;                 // 16-byte vectors per lane per chunk
+constexpr int kChunkVec = 32 * kVec;    // vectors per chunk (1 KB)
 
 struct DispatchArgs {
   const uint8_t* x;
@@ -41,7 +43,7 @@ struct DispatchArgs {
   int32_t chunks;  // chunks per row
 };
 
-__global__ void __launch_bounds__(kThreads, 4) dispatch_kernel(DispatchArgs a) {
+__global__ void __launch_bounds__(kThreads, 8) dispatch_kernel(DispatchArgs a) {
   const int lane = threadIdx.x & 31;
   const int64_t nvec = a.row_bytes >> 4;
   const int64_t n_items = int64_t(a.n) * a.chunks;
@@ -122,7 +124,7 @@ cudaError_t launch_dispatch(const moe_plan& p, int32_t n, const void* x, const f
   a.chunks = int32_t((a.row_bytes / 16 + kChunkVec - 1) / kChunkVec);
   const int sms = num_sms();
   int64_t grid = (int64_t(n) * a.chunks + kWarps - 1) / kWarps;
-  const int64_t cap = int64_t(sms) * 8;
+  const int64_t cap = int64_t(sms) * 16;
   if (grid > cap) grid = cap;
   return launch_pdl(dispatch_kernel, dim3(unsigned(grid)), dim3(kThreads), 0, st, a);
 }

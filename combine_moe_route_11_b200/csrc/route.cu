@@ -190,17 +190,8 @@ cudaError_t launch_coop(const RouteArgs& a, int sms, cudaStream_t st) {
   const int cols = (a.E & 3) == 0 ? a.E / 4 : a.E;
   int grid = a.blocks > cols ? a.blocks : cols;
   if (grid > per_sm[dev] * sms) grid = per_sm[dev] * sms;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(unsigned(grid));
-  cfg.blockDim = dim3(kRouteThreads);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, route_kernel<VPL, VEC>, a);
+  return launch_cooperative(route_kernel<VPL, VEC>, dim3(unsigned(grid)), dim3(kRouteThreads), 0,
+                            st, a);
 }
 
 }  // namespace

@@ -219,17 +219,8 @@ cudaError_t launch_fused(FusedArgs f, int sms, cudaStream_t st) {
   if (grid > int64_t(per_sm[dev]) * sms) grid = int64_t(per_sm[dev]) * sms;
   f.owned = int32_t((int64_t(f.r.n) + grid - 1) / grid);
   if (f.owned > kMaxOwned) return cudaErrorNotSupported;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(unsigned(grid));
-  cfg.blockDim = dim3(kRouteThreads);
-  cfg.dynamicSmemBytes = fused_smem(f.r.blocks, f.r.E, f.owned, f.r.K);
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, f);
+  return launch_cooperative(kernel, dim3(unsigned(grid)), dim3(kRouteThreads),
+                            fused_smem(f.r.blocks, f.r.E, f.owned, f.r.K), st, f);
 }
 
 }  // namespace
