@@ -107,6 +107,18 @@ def test_host_argument_errors_return_before_any_launch(mr):
                             fake, fake, fake, None) == -1          # x not 16-byte aligned
     assert lib.moe_dispatch(p.handle, 0, None, None, None, None, None, None, None, fake,
                             None) == 0                               # n = 0 is a no-op
+    # moe_route_dispatch validates both halves before it launches anything
+    rd = lib.moe_route_dispatch
+    assert rd(p.handle, 65, fake, fake, None, fake, fake, fake, fake, fake, None, fake, fake,
+              fake, None) == -1                                      # n > n_max
+    assert rd(p.handle, 4, fake, fake, None, fake, fake, fake, fake, fake, None, fake, fake,
+              ctypes.c_void_p((1 << 20) + 16), None) == -4          # ws misaligned
+    assert rd(p.handle, 4, fake, fake, None, fake, fake, None, fake, fake, None, fake, fake,
+              fake, None) == -1                                      # no counts
+    assert rd(p.handle, 4, fake, ctypes.c_void_p((1 << 20) + 8), None, fake, fake, fake, fake,
+              fake, None, fake, fake, fake, None) == -1              # x not 16-byte aligned
+    assert rd(p.handle, 4, fake, fake, None, fake, fake, fake, fake, None, None, fake, fake,
+              fake, None) == -1                                      # no recv
     assert lib.moe_combine(p.handle, 65, fake, fake, fake, fake, fake, None) == -1
     assert lib.moe_expert_dequant(p.handle, 4, fake, fake, fake, fake, fake, None) == -2
     assert lib.moe_expert_swiglu(p.handle, 4, fake, fake, fake, fake, fake, fake, fake, fake,
