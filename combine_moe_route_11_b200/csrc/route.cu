@@ -37,6 +37,8 @@
 namespace moe {
 namespace {
 
+static_assert(kWarps == 32, "phase 2 scans one sum per warp with one warp");
+
 // Phase 2 for column unit u (experts [u*W, u*W + W)): rank-major offsets
 // from the expert totals, then the exclusive scan of the unit's count columns
 // over the route blocks into absolute bases.
@@ -58,28 +60,30 @@ __device__ __forceinline__ void scan_column(const RouteArgs& a, int u, const int
     else x += y;
   };
   const V* cnt = reinterpret_cast<const V*>(a.blk);
-  // ---- offsets of this unit's experts from the phase-1 totals: one warp each
-  if (warp < W) {
-    const int e = e0 + warp;
-    const int r = e / per_rank;
-    int sum = 0;
-    for (int e2 = r * per_rank + lane; e2 < e; e2 += 32) sum += __ldcg(tot + e2);
-    sum = __reduce_add_sync(kFull, sum);
-    if (lane == 0) {
-      const int off = r * a.region_rows + sum;
-      s_off[warp] = off;
-      a.expert_off[e] = off;
-      a.counts[e] = __ldcg(tot + e);
-    }
-  }
-  __syncthreads();
-  // ---- exclusive scan of this unit's own columns over the route blocks
+  // ---- this thread's blocks of the unit's count columns, loaded first: they
+  // do not depend on the offsets below
   V* base = reinterpret_cast<V*>(a.bases) + u;
   const V* own = cnt + u;
   const int per = (B + kRouteThreads - 1) / kRouteThreads;
   const int b0 = min(B, tid * per), b1 = min(B, b0 + per);
   V sum = zero;
   for (int b = b0; b < b1; ++b) add(sum, __ldcg(own + int64_t(b) * row));
+  // ---- offsets of this unit's experts from the phase-1 totals: one warp each
+  if (warp < W) {
+    const int e = e0 + warp;
+    const int r = e / per_rank;
+    int tsum = 0;
+    for (int e2 = r * per_rank + lane; e2 < e; e2 += 32) tsum += __ldcg(tot + e2);
+    tsum = __reduce_add_sync(kFull, tsum);
+    if (lane == 0) {
+      const int off = r * a.region_rows + tsum;
+      s_off[warp] = off;
+      a.expert_off[e] = off;
+      a.counts[e] = __ldcg(tot + e);
+    }
+  }
+  // ---- exclusive scan of the columns over the route blocks: within each
+  // warp, then of the warp sums by warp 0
   V incl = sum;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -94,10 +98,29 @@ __device__ __forceinline__ void scan_column(const RouteArgs& a, int u, const int
   }
   if (lane == 31) s_warp[warp] = incl;
   __syncthreads();
+  if (warp == 0) {
+    const V w = s_warp[lane];  // kWarps == 32 warp sums
+    V wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      V y;
+      if constexpr (W == 4) {
+        y.x = __shfl_up_sync(kFull, wi.x, o); y.y = __shfl_up_sync(kFull, wi.y, o);
+        y.z = __shfl_up_sync(kFull, wi.z, o); y.w = __shfl_up_sync(kFull, wi.w, o);
+      } else {
+        y = __shfl_up_sync(kFull, wi, o);
+      }
+      if (lane >= o) add(wi, y);
+    }
+    if constexpr (W == 4) { wi.x -= w.x; wi.y -= w.y; wi.z -= w.z; wi.w -= w.w; }
+    else wi -= w;
+    s_warp[lane] = wi;  // exclusive prefix of the warp sums
+  }
+  __syncthreads();
   V run;
   if constexpr (W == 4) run = make_int4(s_off[0], s_off[1], s_off[2], s_off[3]);
   else run = s_off[0];
-  for (int w = 0; w < warp; ++w) add(run, s_warp[w]);
+  add(run, s_warp[warp]);
   // run + (incl - sum) = absolute base of this thread's first block
   V ex = incl;
   if constexpr (W == 4) { ex.x -= sum.x; ex.y -= sum.y; ex.z -= sum.z; ex.w -= sum.w; }
@@ -105,7 +128,7 @@ __device__ __forceinline__ void scan_column(const RouteArgs& a, int u, const int
   add(run, ex);
   for (int b = b0; b < b1; ++b) {
     base[int64_t(b) * row] = run;
-    add(run, __ldcg(own + int64_t(b) * row));
+    if (b + 1 < b1) add(run, __ldcg(own + int64_t(b) * row));
   }
   __syncthreads();  // shared scratch is reused by the next unit
 }
