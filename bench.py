@@ -281,6 +281,73 @@ def run_reference(args, cfg):
 
 
 # ------------------------------------------------------------------ GPU arm
+def time_e2e(mr, plan, inp, n, out_dtype, dev, stream, steps, world):
+    """Steps through the public moe_layer call, each with the host->device
+    copy of its inputs from pinned memory and the device->host copy of its
+    output.  Two buffer slots let the copies run on their own streams: the
+    copy-in of step i+1 and the copy-out of step i-1 overlap step i's
+    compute (PCIe moves data both ways at once).  Timed with events from the
+    first copy-in to the last copy-out, max over ranks."""
+    lws = plan.new_workspace(dev, layer=True)
+    logits_h = inp["logits"].pin_memory()
+    x_h = inp["x"].pin_memory()
+    xs_h = inp["x_scale"].pin_memory() if inp["x_scale"] is not None else None
+    slots = []
+    for _ in range(2):
+        slots.append({
+            "logits": torch.empty(logits_h.shape, dtype=logits_h.dtype, device=dev),
+            "x": torch.empty(x_h.shape, dtype=x_h.dtype, device=dev),
+            "xs": torch.empty(xs_h.shape, dtype=xs_h.dtype, device=dev) if xs_h is not None
+            else None,
+            "out": torch.empty(n, plan.hidden, dtype=out_dtype, device=dev),
+            "ev_in": torch.cuda.Event(), "ev_comp": torch.cuda.Event(), "ev_out": torch.cuda.Event()})
+    for sl in slots:
+        sl["out_h"] = torch.empty(sl["out"].shape, dtype=sl["out"].dtype).pin_memory()
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+
+    def step(i):
+        sl = slots[i % 2]
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(sl["ev_comp"])  # step i-2 has consumed this slot's inputs
+            sl["logits"].copy_(logits_h, non_blocking=True)
+            sl["x"].copy_(x_h, non_blocking=True)
+            if xs_h is not None:
+                sl["xs"].copy_(xs_h, non_blocking=True)
+            sl["ev_in"].record(s_in)
+        stream.wait_event(sl["ev_in"])
+        if i >= 2:
+            stream.wait_event(sl["ev_out"])  # step i-2's output has left the device
+        mr.moe_layer(plan, sl["logits"], sl["x"], sl["xs"], None, None, sl["out"], lws, stream)
+        sl["ev_comp"].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(sl["ev_comp"])
+            sl["out_h"].copy_(sl["out"], non_blocking=True)
+            sl["ev_out"].record(s_out)
+
+    for i in range(4):
+        step(i)
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s_in)
+    for i in range(steps):
+        step(i)
+    e1.record(s_out)
+    torch.cuda.synchronize(dev)
+    if mr.moe_get_status(plan, lws, stream) != 0:
+        raise RuntimeError("device status set during e2e")
+    e2e_ms = reduce_max(e0.elapsed_time(e1) / steps, dev)
+    h2d = logits_h.numel() * 4 + x_h.numel() * x_h.element_size() + \
+        (xs_h.numel() * 4 if xs_h is not None else 0)
+    d2h = slots[0]["out_h"].numel() * slots[0]["out_h"].element_size()
+    return {"value": world * n / (e2e_ms * 1e-3), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+            "steps": steps, "call": "moe_layer (identity experts)",
+            "pipeline": "two slots: copy-in, moe_layer and copy-out on three streams"}
+
+
 def run_ours(args, cfg):
     world, rank, local = init_dist()
     import combine_moe_route_11_b200 as mr
@@ -414,44 +481,8 @@ def run_ours(args, cfg):
     # ---- end to end through moe_layer with pinned host buffers
     e2e = None
     if not args.no_e2e:
-        lws = plan.new_workspace(dev, layer=True)
-        logits_h = inp["logits"].pin_memory()
-        x_h = inp["x"].pin_memory()
-        xs_h = inp["x_scale"].pin_memory() if inp["x_scale"] is not None else None
-        out_d = torch.empty_like(b["out"])
-        out_h = torch.empty(out_d.shape, dtype=out_d.dtype).pin_memory()
-        logits_d, x_d = torch.empty_like(logits), torch.empty_like(x)
-        xs_d = torch.empty_like(xs) if xs is not None else None
-
-        def e2e_step():
-            logits_d.copy_(logits_h, non_blocking=True)
-            x_d.copy_(x_h, non_blocking=True)
-            if xs_d is not None:
-                xs_d.copy_(xs_h, non_blocking=True)
-            mr.moe_layer(plan, logits_d, x_d, xs_d, None, None, out_d, lws, stream)
-            out_h.copy_(out_d, non_blocking=True)
-
-        e2e_steps = max(3, min(args.steps, 50))
-        for _ in range(3):
-            e2e_step()
-        barrier(dev)
-        torch.cuda.synchronize(dev)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(e2e_steps):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        if mr.moe_get_status(plan, lws, stream) != 0:
-            raise RuntimeError("device status set during e2e")
-        e2e_ms = reduce_max(e0.elapsed_time(e1) / e2e_steps, dev)
-        h2d = logits_h.numel() * 4 + x_h.numel() * x_h.element_size() + \
-            (xs_h.numel() * 4 if xs_h is not None else 0)
-        d2h = out_h.numel() * out_h.element_size()
-        e2e = {"value": world * n / (e2e_ms * 1e-3), "unit": "tokens/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-               "steps": e2e_steps, "call": "moe_layer (identity experts)"}
-        del lws
+        e2e = time_e2e(mr, plan, inp, n, sets[0]["b"]["out"].dtype, dev, stream,
+                       max(3, min(args.steps, 50)), world)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
