@@ -1,8 +1,12 @@
 // C ABI of libmoeroute: plan validation, workspace layout and the entry
 // points declared in include/moeroute.h.  Host code only; every step of the
-// path runs in the kernels of route.cu, dispatch.cu, combine.cu and
-// swiglu_gemm.cu.
+// path runs in the kernels of route.cu, route_dispatch.cu, dispatch.cu,
+// combine.cu, swiglu_gemm.cu and route_noalloc.cu.  The per-device caches
+// here and in the launchers may be reached from several host threads.
 #include "moe_internal.cuh"
+
+#include <atomic>
+#include <mutex>
 
 #include <string.h>
 #include <new>
@@ -10,25 +14,31 @@
 namespace moe {
 
 int num_sms() {
-  static int cached[64] = {0};
+  // per device; a race only computes the same value twice
+  static std::atomic<int> cached[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
-  if (dev < 64 && cached[dev] > 0) return cached[dev];
+  if (dev < 64) {
+    const int c = cached[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
   int v = 0;
   if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
     v = 148;
-  if (dev < 64) cached[dev] = v;
+  if (dev < 64) cached[dev].store(v, std::memory_order_relaxed);
   return v;
 }
 
 cudaError_t set_smem_limit(const void* kernel, int bytes) {
   // (kernel, device) pairs already raised; a handful of kernels, few devices
+  static std::mutex mu;
   static const void* done_k[64];
   static int done_d[64];
   static int done_n = 0;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
   for (int i = 0; i < done_n; ++i)
     if (done_k[i] == kernel && done_d[i] == dev) return cudaSuccess;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);

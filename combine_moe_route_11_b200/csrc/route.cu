@@ -29,6 +29,8 @@
 // deterministic: no atomic decides an order.
 #include "route_common.cuh"
 
+#include <atomic>
+
 #include <float.h>
 #include <limits.h>
 
@@ -198,21 +200,23 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(RouteArgs a) {
 // Cooperative launch: every block resident, as the grid barrier requires.
 template <int VPL, int VEC>
 cudaError_t launch_coop(const RouteArgs& a, int sms, cudaStream_t st) {
-  static int per_sm[64] = {0};  // resident blocks per SM, per device
+  static std::atomic<int> per_sm[64];  // resident blocks per SM, per device (0 = unknown)
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev >= 64) return cudaErrorInvalidDevice;
-  if (per_sm[dev] == 0) {
+  int nb_known = per_sm[dev].load(std::memory_order_relaxed);
+  if (nb_known == 0) {
     int nb = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, route_kernel<VPL, VEC>, kRouteThreads, 0);
     if (e != cudaSuccess) return e;
     if (nb < 1) return cudaErrorInvalidConfiguration;
-    per_sm[dev] = nb;
+    per_sm[dev].store(nb, std::memory_order_relaxed);
+    nb_known = nb;
   }
   const int cols = (a.E & 3) == 0 ? a.E / 4 : a.E;
   int grid = a.blocks > cols ? a.blocks : cols;
-  if (grid > per_sm[dev] * sms) grid = per_sm[dev] * sms;
+  if (grid > nb_known * sms) grid = nb_known * sms;
   return launch_cooperative(route_kernel<VPL, VEC>, dim3(unsigned(grid)), dim3(kRouteThreads), 0,
                             st, a);
 }

@@ -27,6 +27,8 @@
 // Results are identical to moe_route_topk followed by moe_dispatch.
 #include "route_common.cuh"
 
+#include <atomic>
+
 namespace moe {
 namespace {
 
@@ -195,7 +197,7 @@ size_t fused_smem(int blocks, int E, int owned, int K) {
 
 template <int VPL, int VEC>
 cudaError_t launch_fused(FusedArgs f, int sms, cudaStream_t st) {
-  static int per_sm[64] = {0};  // resident blocks per SM, per device
+  static std::atomic<int> per_sm[64];  // resident blocks per SM, per device (0 = unknown)
   // largest use: 32 route blocks of 512 experts, and the picks of up to 64
   // owned tokens of top-k 32 (1024 tokens need a grid of at least 16 blocks)
   constexpr int kMaxOwned = 64;
@@ -207,16 +209,18 @@ cudaError_t launch_fused(FusedArgs f, int sms, cudaStream_t st) {
   if (dev >= 64) return cudaErrorInvalidDevice;
   e = set_smem_limit(reinterpret_cast<const void*>(kernel), kMaxDyn);
   if (e != cudaSuccess) return e;
-  if (per_sm[dev] == 0) {
+  int nb_known = per_sm[dev].load(std::memory_order_relaxed);
+  if (nb_known == 0) {
     int nb = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kernel, kRouteThreads, kMaxDyn);
     if (e != cudaSuccess) return e;
     if (nb < 1) return cudaErrorInvalidConfiguration;
-    per_sm[dev] = nb;
+    per_sm[dev].store(nb, std::memory_order_relaxed);
+    nb_known = nb;
   }
   // one block per token up to the resident limit
   int64_t grid = f.r.n > 1 ? f.r.n : 1;
-  if (grid > int64_t(per_sm[dev]) * sms) grid = int64_t(per_sm[dev]) * sms;
+  if (grid > int64_t(nb_known) * sms) grid = int64_t(nb_known) * sms;
   f.owned = int32_t((int64_t(f.r.n) + grid - 1) / grid);
   if (f.owned > kMaxOwned) return cudaErrorNotSupported;
   return launch_cooperative(kernel, dim3(unsigned(grid)), dim3(kRouteThreads),
