@@ -165,7 +165,9 @@ def test_unfilled_rows_are_never_written():
 
 def test_layer_identity_matches_oracle():
     import combine_moe_route_11_b200 as mr
-    for cfg, n in ((TINY, 64), (C["prefill"], 300), (C["decode"], 128)):
+    # up to 1024 tokens moe_layer routes and dispatches in one launch, above in two
+    for cfg, n in ((TINY, 64), (C["prefill"], 300), (C["decode"], 128),
+                   (C["skewed"].replace(hidden=512), 1500)):
         inp = workloads.make_inputs(cfg, seed=4, n=n)
         inp_np = parity.numpy_inputs(inp)
         ref = oracle.run_path(cfg, inp_np)
