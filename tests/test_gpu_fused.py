@@ -112,3 +112,32 @@ def test_fused_zero_tokens():
     assert mr.moe_get_status(plan, ws) == 0
     assert int(b["counts"].abs().sum()) == 0
     assert int(b["expert_off"].abs().sum()) == 0
+
+
+def test_fused_leaves_unfilled_rows_untouched():
+    """Rows of a region past its filled count are never written by the one-
+    launch path either, and the filled rows are exactly the expert segments."""
+    import combine_moe_route_11_b200 as mr
+    cfg = C["prefill"]
+    n = 300
+    inp = workloads.make_inputs(cfg, seed=8, n=n)
+    plan = mr.Plan.from_config(cfg, n_max=n)
+    dev = torch.device("cuda", 0)
+    ws = plan.new_workspace(dev)
+    b = plan.new_buffers(n, dev)
+    b["recv"].fill_(0xAB)
+    b["recv_scale"].fill_(-3.0)
+    mr.moe_route_dispatch(plan, inp["logits"].cuda(), inp["x"].cuda(), inp["x_scale"].cuda(),
+                          b["topk_idx"], b["topk_w"], b["counts"], b["expert_off"], b["recv"],
+                          b["recv_scale"], b["slot_of"], b["src_of"], ws)
+    assert mr.moe_get_status(plan, ws) == 0
+    filled = torch.zeros(b["recv"].shape[0], dtype=torch.bool, device=dev)
+    filled[b["slot_of"].view(-1).long()] = True
+    assert bool((b["recv"][~filled] == 0xAB).all())
+    assert bool((b["recv_scale"][~filled] == -3.0).all())
+    off = b["expert_off"].cpu().numpy()
+    cnt = b["counts"].cpu().numpy()
+    want = np.zeros(b["recv"].shape[0], bool)
+    for e in range(cfg.n_experts):
+        want[off[e]:off[e] + cnt[e]] = True
+    assert np.array_equal(filled.cpu().numpy(), want)
