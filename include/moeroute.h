@@ -195,8 +195,9 @@ MOE_API moe_status moe_expert_swiglu(const moe_plan* plan, int32_t n, const void
 MOE_API moe_status moe_combine(const moe_plan* plan, int32_t n, const void* y, const float* topk_w,
                        const int32_t* slot_of, void* out, void* ws, moe_stream_t stream);
 
-/* The whole layer on one stream: route -> dispatch -> expert -> combine.
- * Experts are SwiGLU when desc.inter > 0 (w_gate_up, w_down as in
+/* The whole layer on one stream: route -> dispatch -> expert -> combine,
+ * route and dispatch through moe_route_dispatch (one launch up to 1024
+ * tokens).  Experts are SwiGLU when desc.inter > 0 (w_gate_up, w_down as in
  * moe_expert_swiglu), else identity (FP8 rows dequantised, other rows read
  * as Y directly; then y_dtype must equal x_dtype).  logits: device fp32
  * [n, E]; x, x_scale as in moe_dispatch; out: device out_dtype [n, D];
