@@ -141,3 +141,28 @@ def test_fused_leaves_unfilled_rows_untouched():
     for e in range(cfg.n_experts):
         want[off[e]:off[e] + cnt[e]] = True
     assert np.array_equal(filled.cpu().numpy(), want)
+
+
+def test_fused_flags_nonfinite_logit_rows():
+    """A row with fewer than k finite logits sets MOE_ERR_NONFINITE in the
+    one-launch path too; every pick stays a valid expert and every (t, j)
+    still gets a slot, so the dispatched layout stays consistent."""
+    import combine_moe_route_11_b200 as mr
+    cfg = TINY
+    n = 64
+    inp = workloads.make_inputs(cfg, seed=1, n=n)
+    inp["logits"][7, :] = float("nan")
+    inp["logits"][8, 1:] = float("-inf")
+    plan = mr.Plan.from_config(cfg, n_max=n)
+    dev = torch.device("cuda", 0)
+    ws = plan.new_workspace(dev)
+    b = plan.new_buffers(n, dev)
+    mr.moe_route_dispatch(plan, inp["logits"].cuda(), inp["x"].cuda(), None, b["topk_idx"],
+                          b["topk_w"], b["counts"], b["expert_off"], b["recv"], None,
+                          b["slot_of"], b["src_of"], ws)
+    assert mr.moe_get_status(plan, ws) == -7  # MOE_ERR_NONFINITE
+    idx = b["topk_idx"].cpu().numpy()
+    assert ((idx >= 0) & (idx < cfg.n_experts)).all()
+    assert int(b["counts"].sum()) == n * cfg.top_k
+    slots = np.sort(b["slot_of"].cpu().numpy().reshape(-1))
+    assert len(np.unique(slots)) == n * cfg.top_k and slots.min() >= 0
