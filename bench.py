@@ -129,16 +129,52 @@ def recorded_traffic(workload: str):
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    """nvidia-smi samples (SM clock, throttle reasons) while the GPU works."""
+    """SM clock and throttle reasons sampled while the GPU works: through NVML
+    every 10 ms (read-only queries), else `nvidia-smi -lms 100`."""
 
     FIELDS = ["clocks.sm", "clocks.max.sm", "clocks_event_reasons.hw_slowdown",
               "clocks_event_reasons.hw_thermal_slowdown",
               "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    # NVML clock-event reason bits, in the order of NAMES
+    BITS = [0x8, 0x40, 0x20, 0x4]
 
     def __init__(self, device_index: int):
-        self.samples = []
+        self.samples = []  # (time, sm MHz, max MHz, set of reasons)
         self.proc = None
-        self.window = None
+        self.thread = None
+        self.running = False
+        self.source = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            try:
+                nvml_index = torch.cuda._get_nvml_device_index(device_index)
+            except Exception:
+                nvml_index = device_index
+            handle = pynvml.nvmlDeviceGetHandleByIndex(nvml_index)
+            max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM)
+            get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+
+            def poll():
+                while self.running:
+                    try:
+                        mhz = pynvml.nvmlDeviceGetClockInfo(handle, pynvml.NVML_CLOCK_SM)
+                        bits = get_reasons(handle)
+                    except Exception:
+                        break
+                    active = {nm for nm, bit in zip(self.NAMES, self.BITS) if bits & bit}
+                    self.samples.append((time.time(), float(mhz), float(max_mhz), active))
+                    time.sleep(0.01)
+
+            self.running = True
+            self.source = "nvml, 10 ms"
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            self.running = False
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(device_index), "--query-gpu=" + ",".join(self.FIELDS),
@@ -147,47 +183,52 @@ class ClockSampler:
         except OSError:
             self.proc = None
             return
+        self.source = "nvidia-smi, 100 ms"
         self.thread = threading.Thread(target=self._read, daemon=True)
         self.thread.start()
 
     def _read(self):
         for line in self.proc.stdout:
-            self.samples.append((time.time(), line.strip()))
-
-    def wait_first(self, timeout=5.0):
-        t0 = time.time()
-        while self.proc and not self.samples and time.time() - t0 < timeout:
-            time.sleep(0.05)
-
-    def stop(self, t_start: float, t_end: float):
-        if not self.proc:
-            return None
-        time.sleep(0.15)
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ts, line in self.samples:
-            if not (t_start <= ts <= t_end):
-                continue
             parts = [p.strip() for p in line.split(",")]
             if len(parts) != len(self.FIELDS):
                 continue
             try:
-                sm.append(float(parts[0]))
-                mx.append(float(parts[1]))
+                sm, mx = float(parts[0]), float(parts[1])
             except ValueError:
                 continue
-            for nm, v in zip(names, parts[2:]):
-                if v.lower().startswith("active"):
-                    reasons.add(nm)
+            active = {nm for nm, v in zip(self.NAMES, parts[2:]) if v.lower().startswith("active")}
+            self.samples.append((time.time(), sm, mx, active))
+
+    def wait_first(self, timeout=5.0):
+        t0 = time.time()
+        while (self.proc or self.running) and not self.samples and time.time() - t0 < timeout:
+            time.sleep(0.01)
+
+    def stop(self, t_start: float, t_end: float):
+        if self.source is None:
+            return None
+        if self.running:
+            self.running = False
+            self.thread.join(timeout=2)
+        else:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        for ts, mhz, max_mhz, active in list(self.samples):
+            if not (t_start <= ts <= t_end):
+                continue
+            sm.append(mhz)
+            mx.append(max_mhz)
+            reasons |= active
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "source": self.source}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "source": self.source}
 
 
 # ------------------------------------------------------------------ distributed
