@@ -98,6 +98,16 @@ def _stream(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
 
 
+def _ws(plan: "Plan", ws: torch.Tensor, layer: bool = False):
+    """The workspace pointer, after checking the tensor is large enough (the
+    C entry points take no size for it)."""
+    need = plan.layer_workspace_bytes if layer else plan.workspace_bytes
+    if ws.dtype != torch.uint8 or ws.dim() != 1 or ws.numel() < need:
+        raise ValueError(f"ws: need a 1-D uint8 tensor of at least {need} bytes, got "
+                         f"{ws.dtype} {tuple(ws.shape)}")
+    return _ptr(ws)
+
+
 def _expect(t: torch.Tensor, dtypes, shape, name: str):
     if t.dtype not in dtypes:
         raise TypeError(f"{name}: dtype {t.dtype}, expected one of {dtypes}")
@@ -191,7 +201,7 @@ def moe_route_topk(plan: Plan, logits, topk_idx, topk_w, counts, expert_off, ws,
     _expect(counts, (torch.int32,), (plan.n_experts,), "counts")
     _expect(expert_off, (torch.int32,), (plan.n_experts + 1,), "expert_off")
     _check(_lib.moe_route_topk(plan.handle, n, _ptr(logits), _ptr(topk_idx), _ptr(topk_w),
-                               _ptr(counts), _ptr(expert_off), _ptr(ws), _stream(stream)),
+                               _ptr(counts), _ptr(expert_off), _ws(plan, ws), _stream(stream)),
            "moe_route_topk")
 
 
@@ -209,7 +219,7 @@ def moe_dispatch(plan: Plan, x, x_scale, topk_idx, recv, recv_scale, slot_of, sr
     if plan.scale_cols:
         _expect(x_scale, (torch.float32,), (n, plan.scale_cols), "x_scale")
     _check(_lib.moe_dispatch(plan.handle, n, _ptr(x), _ptr(x_scale), _ptr(topk_idx), _ptr(recv),
-                             _ptr(recv_scale), _ptr(slot_of), _ptr(src_of), _ptr(ws),
+                             _ptr(recv_scale), _ptr(slot_of), _ptr(src_of), _ws(plan, ws),
                              _stream(stream)), "moe_dispatch")
 
 
@@ -234,13 +244,13 @@ def moe_route_dispatch(plan: Plan, logits, x, x_scale, topk_idx, topk_w, counts,
     _check(_lib.moe_route_dispatch(plan.handle, n, _ptr(logits), _ptr(x), _ptr(x_scale),
                                    _ptr(topk_idx), _ptr(topk_w), _ptr(counts), _ptr(expert_off),
                                    _ptr(recv), _ptr(recv_scale), _ptr(slot_of), _ptr(src_of),
-                                   _ptr(ws), _stream(stream)), "moe_route_dispatch")
+                                   _ws(plan, ws), _stream(stream)), "moe_route_dispatch")
 
 
 def moe_expert_dequant(plan: Plan, n: int, recv, recv_scale, slot_of, y, ws, stream=None):
     _expect(slot_of, (torch.int32,), (n, plan.top_k), "slot_of")
     _check(_lib.moe_expert_dequant(plan.handle, n, _ptr(recv), _ptr(recv_scale), _ptr(slot_of),
-                                   _ptr(y), _ptr(ws), _stream(stream)), "moe_expert_dequant")
+                                   _ptr(y), _ws(plan, ws), _stream(stream)), "moe_expert_dequant")
 
 
 def moe_expert_swiglu(plan: Plan, n: int, recv, counts, expert_off, w_gate_up, w_down, h, y, ws,
@@ -249,7 +259,7 @@ def moe_expert_swiglu(plan: Plan, n: int, recv, counts, expert_off, w_gate_up, w
     _expect(w_gate_up, (torch.bfloat16,), (E, 2 * I, D), "w_gate_up")
     _expect(w_down, (torch.bfloat16,), (E, D, I), "w_down")
     _check(_lib.moe_expert_swiglu(plan.handle, n, _ptr(recv), _ptr(counts), _ptr(expert_off),
-                                  _ptr(w_gate_up), _ptr(w_down), _ptr(h), _ptr(y), _ptr(ws),
+                                  _ptr(w_gate_up), _ptr(w_down), _ptr(h), _ptr(y), _ws(plan, ws),
                                   _stream(stream)), "moe_expert_swiglu")
 
 
@@ -261,7 +271,7 @@ def moe_combine(plan: Plan, y, topk_w, slot_of, out, ws, stream=None):
     if y.dtype not in _TORCH[plan.y_dtype] or y.shape[-1] != plan.hidden:
         raise TypeError("y: wrong dtype or width")
     _check(_lib.moe_combine(plan.handle, n, _ptr(y), _ptr(topk_w), _ptr(slot_of), _ptr(out),
-                            _ptr(ws), _stream(stream)), "moe_combine")
+                            _ws(plan, ws), _stream(stream)), "moe_combine")
 
 
 def moe_layer(plan: Plan, logits, x, x_scale, w_gate_up, w_down, out, ws, stream=None):
@@ -269,15 +279,14 @@ def moe_layer(plan: Plan, logits, x, x_scale, w_gate_up, w_down, out, ws, stream
     _expect(logits, (torch.float32,), (n, plan.n_experts), "logits")
     _expect(x, _TORCH[plan.x_dtype], (n, plan.hidden), "x")
     _expect(out, _TORCH[plan.out_dtype], (n, plan.hidden), "out")
-    if ws.numel() < plan.layer_workspace_bytes:
-        raise ValueError("ws smaller than moe_layer_workspace_bytes")
     _check(_lib.moe_layer(plan.handle, n, _ptr(logits), _ptr(x), _ptr(x_scale), _ptr(w_gate_up),
-                          _ptr(w_down), _ptr(out), _ptr(ws), _stream(stream)), "moe_layer")
+                          _ptr(w_down), _ptr(out), _ws(plan, ws, layer=True), _stream(stream)),
+           "moe_layer")
 
 
 def moe_layer_buffer(plan: Plan, ws, name: str, dtype, shape) -> torch.Tensor:
     """A view of one intermediate that moe_layer keeps in its workspace."""
-    addr = _lib.moe_layer_buffer(plan.handle, _ptr(ws), name.encode())
+    addr = _lib.moe_layer_buffer(plan.handle, _ws(plan, ws, layer=True), name.encode())
     if not addr:
         raise KeyError(name)
     off = addr - ws.data_ptr()
@@ -290,8 +299,9 @@ def moe_layer_buffer(plan: Plan, ws, name: str, dtype, shape) -> torch.Tensor:
 
 def moe_get_status(plan: Plan, ws, stream=None) -> int:
     """Read and clear the device status word (synchronises the stream)."""
-    return int(_lib.moe_get_status(plan.handle, _ptr(ws), _stream(stream)))
+    return int(_lib.moe_get_status(plan.handle, _ws(plan, ws), _stream(stream)))
 
 
 def moe_workspace_init(plan: Plan, ws, stream=None):
-    _check(_lib.moe_workspace_init(plan.handle, _ptr(ws), _stream(stream)), "moe_workspace_init")
+    _check(_lib.moe_workspace_init(plan.handle, _ws(plan, ws), _stream(stream)),
+           "moe_workspace_init")

@@ -129,3 +129,17 @@ def test_host_argument_errors_return_before_any_launch(mr):
     for code in range(-7, 1):
         assert mr.moe_strerror(code) not in ("", "unknown status")
     p.close()
+
+
+def test_binding_checks_the_workspace_size(mr):
+    """The C entry points take no workspace size, so the binding checks it."""
+    import torch
+    p = mr.Plan(64, 256, 8, 2, 2, "f32", "f32", "f32")
+    small = torch.zeros(p.workspace_bytes - 256, dtype=torch.uint8)
+    with pytest.raises(ValueError):
+        mr.moe_get_status(p, small)
+    with pytest.raises(ValueError):
+        mr.moe_workspace_init(p, torch.zeros(p.workspace_bytes // 4, dtype=torch.int32))
+    with pytest.raises(ValueError):
+        mr._ws(p, torch.zeros(p.workspace_bytes, dtype=torch.uint8), layer=True)
+    p.close()
