@@ -38,6 +38,7 @@ CASES = [
     ("E512", TINY.replace(n_experts=512, top_k=8, n_ranks=8, hidden=128, x_dtype="bf16",
                           y_dtype="bf16", out_dtype="bf16"), 130),
     ("k16", TINY.replace(n_experts=32, top_k=16, n_ranks=2, hidden=64), 100),
+    ("k32_max", TINY.replace(n_experts=64, top_k=32, n_ranks=2, hidden=64), 90),
     ("E512_n128", TINY.replace(n_experts=512, top_k=8, n_ranks=8, hidden=128, x_dtype="bf16",
                                y_dtype="bf16", out_dtype="bf16"), 128),
     # more tokens than resident blocks: blocks own several tokens

@@ -41,6 +41,8 @@ SMALL_CASES = [
     ("bf16_to_f32", C["decode"].replace(hidden=512, out_dtype="f32"), 77),
     ("fp8_small_D", C["prefill"].replace(hidden=256, n_experts=16, top_k=4, n_ranks=4), 129),
     ("k16", TINY.replace(n_experts=32, top_k=16, n_ranks=2, hidden=64), 100),
+    # the largest top-k: one pick per lane of the routing warp
+    ("k32_max", TINY.replace(n_experts=64, top_k=32, n_ranks=2, hidden=64), 90),
 ]
 
 
