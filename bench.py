@@ -691,7 +691,8 @@ def main(argv=None):
     ap.add_argument("--graph", action="store_true",
                     help="replay each step as one captured CUDA graph")
     ap.add_argument("--tokens", type=int, default=0,
-                    help="override N (smaller batches for profiler captures only)")
+                    help="override N (smaller batches for profiler captures, larger ones for "
+                         "the supplementary tensor-bound layer runs)")
     ap.add_argument("--experts", type=int, default=0,
                     help="override E (smaller weight sets for profiler captures only)")
     args = ap.parse_args(argv)
