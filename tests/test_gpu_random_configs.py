@@ -21,7 +21,7 @@ import workloads
 pytestmark = pytest.mark.gpu
 
 
-def _random_configs(count=24, seed=2027):
+def _random_configs(count=48, seed=2027):
     rng = random.Random(seed)
     base = workloads.CONFIGS["tiny"]
     out = []
