@@ -130,7 +130,9 @@ def recorded_traffic(workload: str):
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     """SM clock and throttle reasons sampled while the GPU works: through NVML
-    every 10 ms (read-only queries), else `nvidia-smi -lms 100`."""
+    every 2 ms (read-only queries; the calls release the GIL), else
+    `nvidia-smi -lms 100`.  A timed region shorter than the period reports the
+    samples nearest to it and says so."""
 
     FIELDS = ["clocks.sm", "clocks.max.sm", "clocks_event_reasons.hw_slowdown",
               "clocks_event_reasons.hw_thermal_slowdown",
@@ -166,10 +168,10 @@ class ClockSampler:
                         break
                     active = {nm for nm, bit in zip(self.NAMES, self.BITS) if bits & bit}
                     self.samples.append((time.time(), float(mhz), float(max_mhz), active))
-                    time.sleep(0.01)
+                    time.sleep(0.002)
 
             self.running = True
-            self.source = "nvml, 10 ms"
+            self.source = "nvml, 2 ms"
             self.thread = threading.Thread(target=poll, daemon=True)
             self.thread.start()
             return
@@ -217,18 +219,24 @@ class ClockSampler:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-        sm, mx, reasons = [], [], set()
-        for ts, mhz, max_mhz, active in list(self.samples):
-            if not (t_start <= ts <= t_end):
-                continue
-            sm.append(mhz)
-            mx.append(max_mhz)
-            reasons |= active
-        if not sm:
+        all_samples = list(self.samples)
+        window = [x for x in all_samples if t_start <= x[0] <= t_end]
+        where = "during the timed region"
+        if not window and all_samples:
+            # a region shorter than the period: the samples closest to it
+            mid = 0.5 * (t_start + t_end)
+            window = sorted(all_samples, key=lambda x: abs(x[0] - mid))[:2]
+            where = "nearest to the timed region (shorter than the sampling period)"
+        if not window:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
                     "source": self.source}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
-                "reasons": sorted(reasons), "samples": len(sm), "source": self.source}
+        sm = [x[1] for x in window]
+        reasons = set()
+        for x in window:
+            reasons |= x[3]
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(x[2] for x in window),
+                "reasons": sorted(reasons), "samples": len(sm), "source": self.source,
+                "window": where}
 
 
 # ------------------------------------------------------------------ distributed
