@@ -130,7 +130,7 @@ def recorded_traffic(workload: str):
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     """SM clock and throttle reasons sampled while the GPU works: through NVML
-    every 2 ms (read-only queries; the calls release the GIL), else
+    every 5 ms (read-only queries; the calls release the GIL), else
     `nvidia-smi -lms 100`.  A timed region shorter than the period reports the
     samples nearest to it and says so."""
 
@@ -168,10 +168,10 @@ class ClockSampler:
                         break
                     active = {nm for nm, bit in zip(self.NAMES, self.BITS) if bits & bit}
                     self.samples.append((time.time(), float(mhz), float(max_mhz), active))
-                    time.sleep(0.002)
+                    time.sleep(0.005)
 
             self.running = True
-            self.source = "nvml, 2 ms"
+            self.source = "nvml, 5 ms"
             self.thread = threading.Thread(target=poll, daemon=True)
             self.thread.start()
             return
