@@ -131,6 +131,10 @@ class Plan:
         h = _P()
         _check(_lib.moe_plan_create(ctypes.byref(d), ctypes.byref(h)), "moe_plan_create")
         self._h = h
+        # constant for the plan's lifetime: asked once, not on every call
+        self._ws_bytes = int(_lib.moe_workspace_bytes(h))
+        self._layer_ws_bytes = int(_lib.moe_layer_workspace_bytes(h))
+        self._recv_rows = {}
 
     @classmethod
     def from_config(cls, cfg, n_max: int | None = None) -> "Plan":
@@ -154,17 +158,20 @@ class Plan:
 
     @property
     def workspace_bytes(self) -> int:
-        return int(_lib.moe_workspace_bytes(self._h))
+        return self._ws_bytes
 
     @property
     def layer_workspace_bytes(self) -> int:
-        return int(_lib.moe_layer_workspace_bytes(self._h))
+        return self._layer_ws_bytes
 
     def region_rows(self, n: int) -> int:
         return int(_lib.moe_region_rows(self._h, n))
 
     def recv_rows(self, n: int) -> int:
-        return int(_lib.moe_recv_rows(self._h, n))
+        rows = self._recv_rows.get(n)
+        if rows is None:
+            rows = self._recv_rows[n] = int(_lib.moe_recv_rows(self._h, n))
+        return rows
 
     def new_workspace(self, device="cuda", layer: bool = False) -> torch.Tensor:
         nbytes = self.layer_workspace_bytes if layer else self.workspace_bytes
