@@ -106,10 +106,17 @@ def read_peaks() -> tuple[float, str]:
 
 
 def kernel_source_hash() -> str:
+    """Hash of the source the combine kernel is compiled from: combine.cu and
+    the device-helper part of the internal header (host-side declarations
+    there do not change the kernel)."""
     h = hashlib.sha256()
-    for name in ("combine.cu", "moe_internal.cuh"):
-        with open(os.path.join(ROOT, "combine_moe_route_11_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+    csrc = os.path.join(ROOT, "combine_moe_route_11_b200", "csrc")
+    with open(os.path.join(csrc, "combine.cu"), "rb") as f:
+        h.update(f.read())
+    with open(os.path.join(csrc, "moe_internal.cuh"), "rb") as f:
+        text = f.read()
+    marker = b"// ------------------------------------------------------------------ device helpers"
+    h.update(text[text.find(marker):] if marker in text else text)
     return h.hexdigest()[:16]
 
 

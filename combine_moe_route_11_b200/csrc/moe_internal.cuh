@@ -30,9 +30,6 @@ struct Ctrl {
 };
 static_assert(sizeof(Ctrl) == 256, "control block is 256 bytes");
 
-__host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
-__host__ __device__ __forceinline__ int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
-
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 inline int elem_bytes(int dtype) {
@@ -219,7 +216,7 @@ __device__ __forceinline__ void st_cs_v4(void* p, const uint4& v) {
                : "memory");
 }
 
-// ---- bulk asynchronous copies (TMA engine) and mbarriers, no multicast
+// ---- mbarriers (for the tensor-memory-accelerator copies of the grouped GEMM)
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -232,12 +229,6 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
 // Make mbarrier initialisation visible to the async proxy.
 __device__ __forceinline__ void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-
-// Order this thread's generic-proxy shared-memory accesses before later
-// async-proxy (bulk copy) accesses of the same bytes, and vice versa.
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
@@ -270,39 +261,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   while (!mbar_try_wait(bar, parity))
     if (clock64() - t0 > (1ll << 31)) return false;
   return true;
-}
-
-// global -> shared bulk copy completing on an mbarrier (bytes % 16 == 0,
-// both addresses 16-byte aligned).
-__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes,
-                                          uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-          "r"(smem_addr(smem_dst)),
-      "l"(gsrc), "r"(bytes), "r"(smem_addr(bar))
-      : "memory");
-}
-
-// shared -> global bulk copy tracked by this thread's bulk groups.
-__device__ __forceinline__ void bulk_store(void* gdst, const void* smem_src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
-               "r"(smem_addr(smem_src)), "r"(bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ void bulk_commit() {
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-
-// Wait until at most N of this thread's bulk groups still read shared memory.
-template <int N>
-__device__ __forceinline__ void bulk_wait_read() {
-  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
-}
-
-// Wait until all of this thread's bulk groups have completed.
-__device__ __forceinline__ void bulk_wait_all() {
-  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
