@@ -77,7 +77,7 @@ typedef struct CUstream_st* moe_stream_t;
 typedef enum {
   MOE_OK = 0,
   MOE_ERR_INVALID_ARG = -1,   /* bad pointer, size, alignment or n > n_max */
-  MOE_ERR_UNSUPPORTED = -2,   /* valid but outside what this build implements */
+  MOE_ERR_UNSUPPORTED = -2,   /* valid but outside what this library implements */
   MOE_ERR_CUDA = -3,          /* a CUDA runtime call or launch failed */
   MOE_ERR_WORKSPACE = -4,     /* workspace too small or misaligned */
   MOE_ERR_DEVICE_INDEX = -5,  /* device saw an expert id or slot out of range */
