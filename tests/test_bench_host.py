@@ -77,3 +77,30 @@ def test_fused_batch_limit_agrees_with_the_library():
     assert bench.FUSED_MAX_TOKENS == mr.FUSED_MAX_TOKENS == 32 * 32
     with open(os.path.join(ROOT, "include", "moeroute.h")) as f:
         assert "n <= 1024 tokens" in f.read()
+
+
+def test_clock_sampler_window_and_short_region_fallback():
+    """Samples inside the timed region decide the clock record; a region
+    shorter than the sampling period reports the nearest samples and says so.
+    Reasons seen in any sample of the window are reported."""
+    sys.path.insert(0, ROOT)
+    import bench
+    s = bench.ClockSampler.__new__(bench.ClockSampler)
+    s.running, s.proc, s.thread, s.source = False, None, None, "test"
+    s.samples = [(1.00, 1965.0, 1965.0, set()), (1.01, 1410.0, 1965.0, {"sw_power_cap"}),
+                 (1.02, 1400.0, 1965.0, {"sw_power_cap"}), (1.05, 1965.0, 1965.0, set())]
+
+    class _Proc:  # stands in for the nvidia-smi child that stop() ends
+        def terminate(self):
+            pass
+
+        def wait(self, timeout=None):
+            return 0
+
+    s.proc = _Proc()
+    rec = s.stop(1.005, 1.025)
+    assert rec["samples"] == 2 and rec["sm_mhz"] == 1405.0
+    assert rec["reasons"] == ["sw_power_cap"] and rec["window"] == "during the timed region"
+    s.proc = _Proc()
+    rec = s.stop(1.031, 1.032)  # between samples: the two nearest
+    assert rec["samples"] == 2 and rec["window"].startswith("nearest")
