@@ -105,31 +105,48 @@ def read_peaks() -> tuple[float, str]:
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def _device_part(name: str, start: bytes = b"", end: bytes = b"") -> bytes:
+    """The bytes of a source file between two markers (whole ends if absent)."""
+    with open(os.path.join(ROOT, "combine_moe_route_11_b200", "csrc", name), "rb") as f:
+        text = f.read()
+    a = text.find(start) if start and start in text else 0
+    b = text.find(end) if end and end in text else len(text)
+    return text[a:b]
+
+
+_HELPERS = b"// ------------------------------------------------------------------ device helpers"
+
+
 def kernel_source_hash() -> str:
     """Hash of the source the combine kernel is compiled from: combine.cu and
     the device-helper part of the internal header (host-side declarations
     there do not change the kernel)."""
     h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "combine_moe_route_11_b200", "csrc")
-    with open(os.path.join(csrc, "combine.cu"), "rb") as f:
-        h.update(f.read())
-    with open(os.path.join(csrc, "moe_internal.cuh"), "rb") as f:
-        text = f.read()
-    marker = b"// ------------------------------------------------------------------ device helpers"
-    h.update(text[text.find(marker):] if marker in text else text)
+    h.update(_device_part("combine.cu"))
+    h.update(_device_part("moe_internal.cuh", start=_HELPERS))
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload: str):
-    """DRAM bytes per combine launch from the committed ncu summary, if it was
-    taken on the current kernel source (else None)."""
+def gemm_source_hash() -> str:
+    """Hash of the device code of the grouped GEMM kernels: swiglu_gemm.cu up to
+    its host side, and the device-helper part of the internal header."""
+    h = hashlib.sha256()
+    h.update(_device_part("swiglu_gemm.cu",
+                          end=b"// ---------------------------------------------------------------- host side"))
+    h.update(_device_part("moe_internal.cuh", start=_HELPERS))
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str, source_hash=kernel_source_hash):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary, if it was taken on the current kernel source (else None)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
             rec = json.load(f).get(workload)
     except (OSError, ValueError):
         return None
-    if not rec or rec.get("source_hash") != kernel_source_hash():
+    if not rec or rec.get("source_hash") != source_hash():
         return None
     return rec.get("dram_bytes_per_launch")
 
@@ -665,10 +682,14 @@ def run_layer(args, cfg):
                    "achieved": tfs, "peak": peak,
                    "peak_kind": "measured sustained" if peaks else "fallback",
                    "unit": "TFLOP/s", "frac": tfs / peak, "traffic": None}
+    full_shape = (n, E, D, I) == (workloads.CONFIGS["layer"].n, workloads.CONFIGS["layer"].n_experts,
+                                  workloads.CONFIGS["layer"].hidden,
+                                  workloads.CONFIGS["layer"].inter)
     hbm_line = {"bound": "hbm", "kernel": "expert_gemm (GEMM1 + GEMM2)",
                 "achieved": gbs, "peak": hbm_peak,
                 "peak_kind": "measured" if peaks else "fallback",
-                "unit": "GB/s", "frac": gbs / hbm_peak, "traffic": None,
+                "unit": "GB/s", "frac": gbs / hbm_peak,
+                "traffic": recorded_traffic("layer", gemm_source_hash) if full_shape else None,
                 "algorithmic_bytes": wbytes + abytes}
     hbm_bound = (wbytes + abytes) / (hbm_peak * 1e9) >= flops / (peak * 1e12)
     roofline, other = (hbm_line, tensor_line) if hbm_bound else (tensor_line, hbm_line)
