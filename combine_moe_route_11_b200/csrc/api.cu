@@ -272,9 +272,20 @@ moe_status moe_layer(const moe_plan* p, int32_t n, const float* logits, const vo
   moe_status s = check_call(p, n, ws);
   if (s != MOE_OK) return s;
   const moe_desc& d = p->d;
+  // Every argument error is found here, before the first launch: the stages
+  // below only receive pointers into ws (256-byte aligned by the layout) or
+  // arguments checked here, so none of them can reject the call halfway.
   if (d.inter == 0 && d.x_dtype != MOE_FP8_E4M3 && d.y_dtype != d.x_dtype)
     return MOE_ERR_UNSUPPORTED;
+  if (d.inter == 0 && d.x_dtype == MOE_FP8_E4M3 && d.y_dtype != MOE_BF16)
+    return MOE_ERR_UNSUPPORTED;  // the FP8 identity expert writes bf16
   if (d.inter > 0 && (!w_gate_up || !w_down)) return MOE_ERR_INVALID_ARG;
+  if (n > 0) {
+    if (!logits || !x || !out) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(logits) || !aligned16(x) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+    if (p->scale_cols > 0 && !x_scale) return MOE_ERR_INVALID_ARG;
+    if (d.inter > 0 && (!aligned16(w_gate_up) || !aligned16(w_down))) return MOE_ERR_INVALID_ARG;
+  }
   char* b = static_cast<char*>(ws);
   const Layout& L = p->lay;
   int32_t* topk_idx = reinterpret_cast<int32_t*>(b + L.topk_idx);

@@ -170,7 +170,8 @@ MOE_API moe_status moe_route_dispatch(const moe_plan* plan, int32_t n, const flo
  * c / scale_block]) for every filled slot s = slot_of[t, j], correctly rounded
  * (to nearest even) from the exact product.  recv: device e4m3 [T, D];
  * recv_scale: device fp32 [T, D/scale_block] (NULL = scale 1); y: device
- * y_dtype [T, D]. */
+ * bf16 [T, D].  Plans whose x_dtype is not FP8 or whose y_dtype is not BF16
+ * get MOE_ERR_UNSUPPORTED. */
 MOE_API moe_status moe_expert_dequant(const moe_plan* plan, int32_t n, const void* recv,
                               const float* recv_scale, const int32_t* slot_of, void* y,
                               void* ws, moe_stream_t stream);
@@ -198,11 +199,13 @@ MOE_API moe_status moe_combine(const moe_plan* plan, int32_t n, const void* y, c
 /* The whole layer on one stream: route -> dispatch -> expert -> combine,
  * route and dispatch through moe_route_dispatch (one launch up to 1024
  * tokens).  Experts are SwiGLU when desc.inter > 0 (w_gate_up, w_down as in
- * moe_expert_swiglu), else identity (FP8 rows dequantised, other rows read
- * as Y directly; then y_dtype must equal x_dtype).  logits: device fp32
+ * moe_expert_swiglu), else identity (FP8 rows dequantised to bf16, so then
+ * y_dtype must be BF16; other rows read as Y directly, so then y_dtype must
+ * equal x_dtype; MOE_ERR_UNSUPPORTED otherwise).  logits: device fp32
  * [n, E]; x, x_scale as in moe_dispatch; out: device out_dtype [n, D];
  * ws: moe_layer_workspace_bytes() of zero-filled device memory, which holds
- * every intermediate (see moe_layer_buffer). */
+ * every intermediate (see moe_layer_buffer).  Every argument error is
+ * returned before the first stage is enqueued. */
 MOE_API moe_status moe_layer(const moe_plan* plan, int32_t n, const float* logits, const void* x,
                      const float* x_scale, const void* w_gate_up, const void* w_down,
                      void* out, void* ws, moe_stream_t stream);

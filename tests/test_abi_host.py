@@ -131,6 +131,29 @@ def test_host_argument_errors_return_before_any_launch(mr):
     p.close()
 
 
+def test_layer_rejects_bad_arguments_before_its_first_stage(mr):
+    """moe_layer checks every argument that a later stage would reject before
+    it enqueues route and dispatch.  Without a GPU any launch fails with
+    MOE_ERR_CUDA (-3), so the host-side codes below show that no stage ran."""
+    fake = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    lib = mr._lib
+    # FP8 rows with identity experts dequantise to bf16: an fp32 Y is unsupported
+    p = mr.Plan(64, 256, 8, 2, 2, "fp8_e4m3", "f32", "f32", scale_block=128)
+    assert lib.moe_layer(p.handle, 4, fake, fake, fake, None, None, fake, fake, None) == -2
+    p.close()
+    p = mr.Plan(64, 256, 8, 2, 2, "fp8_e4m3", "bf16", "bf16", scale_block=128)
+    assert lib.moe_layer(p.handle, 4, fake, fake, None, None, None, fake, fake, None) == -1
+    assert lib.moe_layer(p.handle, 4, fake, fake, fake, None, None, None, fake, None) == -1
+    assert lib.moe_layer(p.handle, 4, fake, fake, fake, None, None, odd, fake, None) == -1
+    assert lib.moe_layer(p.handle, 4, odd, fake, fake, None, None, fake, fake, None) == -1
+    p.close()
+    p = mr.Plan(64, 256, 8, 2, 2, "bf16", "bf16", "bf16", inter=128)
+    assert lib.moe_layer(p.handle, 4, fake, fake, None, None, fake, fake, fake, None) == -1
+    assert lib.moe_layer(p.handle, 4, fake, fake, None, fake, odd, fake, fake, None) == -1
+    p.close()
+
+
 def test_binding_checks_the_workspace_size(mr):
     """The C entry points take no workspace size, so the binding checks it."""
     import torch
