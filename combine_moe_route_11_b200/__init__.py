@@ -14,9 +14,10 @@ import os
 import torch
 
 __all__ = [
-    "MoeError", "Plan", "LIB_PATH", "moe_route_topk", "moe_dispatch", "moe_expert_dequant",
-    "moe_expert_swiglu", "moe_combine", "moe_layer", "moe_layer_buffer", "moe_get_status",
-    "moe_workspace_init", "moe_strerror", "DTYPE_CODES", "ELEM_BYTES",
+    "MoeError", "Plan", "LIB_PATH", "moe_route_topk", "moe_dispatch", "moe_route_dispatch",
+    "moe_expert_dequant", "moe_expert_swiglu", "moe_combine", "moe_layer", "moe_layer_buffer",
+    "moe_get_status", "moe_workspace_init", "moe_strerror", "DTYPE_CODES", "ELEM_BYTES",
+    "FUSED_MAX_TOKENS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoeroute.so")
@@ -109,10 +110,33 @@ def _ws(plan: "Plan", ws: torch.Tensor, layer: bool = False):
 
 
 def _expect(t: torch.Tensor, dtypes, shape, name: str):
+    if t is None:
+        raise ValueError(f"{name}: required")
     if t.dtype not in dtypes:
         raise TypeError(f"{name}: dtype {t.dtype}, expected one of {dtypes}")
     if tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _expect_rows(t: torch.Tensor, dtypes, rows: int, width: int, name: str):
+    """A [>= rows, width] buffer indexed by slot: the kernels reach any row
+    below T, so a shorter tensor would be written or read out of bounds."""
+    if t is None:
+        raise ValueError(f"{name}: required")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected one of {dtypes}")
+    if t.dim() != 2 or t.shape[0] < rows or t.shape[1] != width:
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, need at least ({rows}, {width})")
+
+
+def _expect_scales(plan: "Plan", t, rows: int, name: str, exact: bool = False):
+    """fp32 per-block scales of FP8 rows; ignored (may be None) without them."""
+    if not plan.scale_cols:
+        return
+    if exact:
+        _expect(t, (torch.float32,), (rows, plan.scale_cols), name)
+    else:
+        _expect_rows(t, (torch.float32,), rows, plan.scale_cols, name)
 
 
 class Plan:
@@ -212,19 +236,23 @@ def moe_route_topk(plan: Plan, logits, topk_idx, topk_w, counts, expert_off, ws,
            "moe_route_topk")
 
 
+def _check_dispatch_outputs(plan: Plan, T: int, x_scale, n: int, recv, recv_scale, slot_of,
+                            src_of):
+    _expect_rows(recv, _TORCH[plan.x_dtype], T, plan.hidden, "recv")
+    _expect(slot_of, (torch.int32,), (n, plan.top_k), "slot_of")
+    if src_of is None or src_of.dtype != torch.int32 or src_of.dim() != 1 or src_of.shape[0] < T:
+        raise ValueError(f"src_of: need a 1-D int32 tensor of at least {T} entries")
+    _expect_scales(plan, x_scale, n, "x_scale", exact=True)
+    _expect_scales(plan, recv_scale, T, "recv_scale")
+
+
 def moe_dispatch(plan: Plan, x, x_scale, topk_idx, recv, recv_scale, slot_of, src_of, ws,
                  stream=None):
     n = x.shape[0]
     T = plan.recv_rows(n)
     _expect(x, _TORCH[plan.x_dtype], (n, plan.hidden), "x")
     _expect(topk_idx, (torch.int32,), (n, plan.top_k), "topk_idx")
-    if recv.shape[0] < T or tuple(recv.shape[1:]) != (plan.hidden,):
-        raise ValueError(f"recv: shape {tuple(recv.shape)}, need at least ({T}, {plan.hidden})")
-    _expect(slot_of, (torch.int32,), (n, plan.top_k), "slot_of")
-    if src_of.shape[0] < T:
-        raise ValueError("src_of too short")
-    if plan.scale_cols:
-        _expect(x_scale, (torch.float32,), (n, plan.scale_cols), "x_scale")
+    _check_dispatch_outputs(plan, T, x_scale, n, recv, recv_scale, slot_of, src_of)
     _check(_lib.moe_dispatch(plan.handle, n, _ptr(x), _ptr(x_scale), _ptr(topk_idx), _ptr(recv),
                              _ptr(recv_scale), _ptr(slot_of), _ptr(src_of), _ws(plan, ws),
                              _stream(stream)), "moe_dispatch")
@@ -241,13 +269,7 @@ def moe_route_dispatch(plan: Plan, logits, x, x_scale, topk_idx, topk_w, counts,
     _expect(topk_w, (torch.float32,), (n, plan.top_k), "topk_w")
     _expect(counts, (torch.int32,), (plan.n_experts,), "counts")
     _expect(expert_off, (torch.int32,), (plan.n_experts + 1,), "expert_off")
-    if recv.shape[0] < T or tuple(recv.shape[1:]) != (plan.hidden,):
-        raise ValueError(f"recv: shape {tuple(recv.shape)}, need at least ({T}, {plan.hidden})")
-    _expect(slot_of, (torch.int32,), (n, plan.top_k), "slot_of")
-    if src_of.shape[0] < T:
-        raise ValueError("src_of too short")
-    if plan.scale_cols:
-        _expect(x_scale, (torch.float32,), (n, plan.scale_cols), "x_scale")
+    _check_dispatch_outputs(plan, T, x_scale, n, recv, recv_scale, slot_of, src_of)
     _check(_lib.moe_route_dispatch(plan.handle, n, _ptr(logits), _ptr(x), _ptr(x_scale),
                                    _ptr(topk_idx), _ptr(topk_w), _ptr(counts), _ptr(expert_off),
                                    _ptr(recv), _ptr(recv_scale), _ptr(slot_of), _ptr(src_of),
@@ -255,7 +277,12 @@ def moe_route_dispatch(plan: Plan, logits, x, x_scale, topk_idx, topk_w, counts,
 
 
 def moe_expert_dequant(plan: Plan, n: int, recv, recv_scale, slot_of, y, ws, stream=None):
+    T = plan.recv_rows(n)
     _expect(slot_of, (torch.int32,), (n, plan.top_k), "slot_of")
+    _expect_rows(recv, _TORCH["fp8_e4m3"], T, plan.hidden, "recv")
+    if recv_scale is not None:
+        _expect_scales(plan, recv_scale, T, "recv_scale")
+    _expect_rows(y, (torch.bfloat16,), T, plan.hidden, "y")
     _check(_lib.moe_expert_dequant(plan.handle, n, _ptr(recv), _ptr(recv_scale), _ptr(slot_of),
                                    _ptr(y), _ws(plan, ws), _stream(stream)), "moe_expert_dequant")
 
@@ -263,8 +290,14 @@ def moe_expert_dequant(plan: Plan, n: int, recv, recv_scale, slot_of, y, ws, str
 def moe_expert_swiglu(plan: Plan, n: int, recv, counts, expert_off, w_gate_up, w_down, h, y, ws,
                       stream=None):
     E, D, I = plan.n_experts, plan.hidden, plan.inter
+    T = plan.recv_rows(n)
     _expect(w_gate_up, (torch.bfloat16,), (E, 2 * I, D), "w_gate_up")
     _expect(w_down, (torch.bfloat16,), (E, D, I), "w_down")
+    _expect_rows(recv, (torch.bfloat16,), T, D, "recv")
+    _expect(counts, (torch.int32,), (E,), "counts")
+    _expect(expert_off, (torch.int32,), (E + 1,), "expert_off")
+    _expect_rows(h, (torch.bfloat16,), T, I, "h")
+    _expect_rows(y, (torch.bfloat16,), T, D, "y")
     _check(_lib.moe_expert_swiglu(plan.handle, n, _ptr(recv), _ptr(counts), _ptr(expert_off),
                                   _ptr(w_gate_up), _ptr(w_down), _ptr(h), _ptr(y), _ws(plan, ws),
                                   _stream(stream)), "moe_expert_swiglu")
@@ -275,8 +308,7 @@ def moe_combine(plan: Plan, y, topk_w, slot_of, out, ws, stream=None):
     _expect(out, _TORCH[plan.out_dtype], (n, plan.hidden), "out")
     _expect(topk_w, (torch.float32,), (n, plan.top_k), "topk_w")
     _expect(slot_of, (torch.int32,), (n, plan.top_k), "slot_of")
-    if y.dtype not in _TORCH[plan.y_dtype] or y.shape[-1] != plan.hidden:
-        raise TypeError("y: wrong dtype or width")
+    _expect_rows(y, _TORCH[plan.y_dtype], plan.recv_rows(n), plan.hidden, "y")
     _check(_lib.moe_combine(plan.handle, n, _ptr(y), _ptr(topk_w), _ptr(slot_of), _ptr(out),
                             _ws(plan, ws), _stream(stream)), "moe_combine")
 
@@ -286,6 +318,11 @@ def moe_layer(plan: Plan, logits, x, x_scale, w_gate_up, w_down, out, ws, stream
     _expect(logits, (torch.float32,), (n, plan.n_experts), "logits")
     _expect(x, _TORCH[plan.x_dtype], (n, plan.hidden), "x")
     _expect(out, _TORCH[plan.out_dtype], (n, plan.hidden), "out")
+    _expect_scales(plan, x_scale, n, "x_scale", exact=True)
+    if plan.inter > 0:
+        E, D, I = plan.n_experts, plan.hidden, plan.inter
+        _expect(w_gate_up, (torch.bfloat16,), (E, 2 * I, D), "w_gate_up")
+        _expect(w_down, (torch.bfloat16,), (E, D, I), "w_down")
     _check(_lib.moe_layer(plan.handle, n, _ptr(logits), _ptr(x), _ptr(x_scale), _ptr(w_gate_up),
                           _ptr(w_down), _ptr(out), _ws(plan, ws, layer=True), _stream(stream)),
            "moe_layer")
@@ -301,6 +338,8 @@ def moe_layer_buffer(plan: Plan, ws, name: str, dtype, shape) -> torch.Tensor:
     for s in shape:
         count *= s
     nbytes = count * torch.empty((), dtype=dtype).element_size()
+    if off < 0 or off + nbytes > ws.numel():
+        raise ValueError(f"{name}: {nbytes} bytes at offset {off} exceed the workspace")
     return ws[off:off + nbytes].view(dtype).view(*shape)
 
 

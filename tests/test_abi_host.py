@@ -166,3 +166,72 @@ def test_binding_checks_the_workspace_size(mr):
     with pytest.raises(ValueError):
         mr._ws(p, torch.zeros(p.workspace_bytes, dtype=torch.uint8), layer=True)
     p.close()
+
+
+def test_binding_checks_slot_indexed_buffers(mr):
+    """Buffers indexed by slot must hold T rows of the plan's width and dtype:
+    the binding rejects shorter or mistyped tensors before any pointer reaches
+    the library.  The tensors here are on the CPU, so a call that passes every
+    check stops at the binding's CUDA-tensor check instead."""
+    import torch
+    n = 16
+    p = mr.Plan(64, 256, 8, 2, 2, "bf16", "bf16", "bf16")
+    T = p.recv_rows(n)
+    ws = torch.zeros(p.workspace_bytes, dtype=torch.uint8)
+    w = torch.zeros(n, 2)
+    so = torch.zeros(n, 2, dtype=torch.int32)
+    out = torch.zeros(n, 256, dtype=torch.bfloat16)
+    bf = lambda r, c=256: torch.zeros(r, c, dtype=torch.bfloat16)  # noqa: E731
+    with pytest.raises(ValueError, match="need at least"):
+        mr.moe_combine(p, bf(T - 1), w, so, out, ws)
+    with pytest.raises(TypeError, match="y: dtype"):
+        mr.moe_combine(p, torch.zeros(T, 256), w, so, out, ws)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        mr.moe_combine(p, bf(T), w, so, out, ws)
+    x = bf(n)
+    idx = torch.zeros(n, 2, dtype=torch.int32)
+    src = torch.zeros(T, dtype=torch.int32)
+    with pytest.raises(ValueError, match="recv: shape"):
+        mr.moe_dispatch(p, x, None, idx, bf(T, 128), None, so, src, ws)
+    with pytest.raises(TypeError, match="recv: dtype"):
+        mr.moe_dispatch(p, x, None, idx, torch.zeros(T, 256, dtype=torch.uint8), None, so, src, ws)
+    with pytest.raises(ValueError, match="src_of"):
+        mr.moe_dispatch(p, x, None, idx, bf(T), None, so, src[:-1], ws)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        mr.moe_dispatch(p, x, None, idx, bf(T), None, so, src, ws)
+    p.close()
+
+    p = mr.Plan(64, 256, 8, 2, 2, "fp8_e4m3", "bf16", "bf16", scale_block=128)
+    T = p.recv_rows(n)
+    ws = torch.zeros(p.layer_workspace_bytes, dtype=torch.uint8)
+    q = lambda r: torch.zeros(r, 256, dtype=torch.uint8)  # noqa: E731
+    xs = torch.ones(n, 2)
+    with pytest.raises(ValueError, match="recv_scale"):
+        mr.moe_dispatch(p, q(n), xs, idx, q(T), torch.ones(T - 1, 2), so, src, ws)
+    with pytest.raises(ValueError, match="x_scale: required"):
+        mr.moe_dispatch(p, q(n), None, idx, q(T), torch.ones(T, 2), so, src, ws)
+    with pytest.raises(TypeError, match="y: dtype"):
+        mr.moe_expert_dequant(p, n, q(T), torch.ones(T, 2), so, torch.zeros(T, 256), ws)
+    with pytest.raises(ValueError, match="y: shape"):
+        mr.moe_expert_dequant(p, n, q(T), torch.ones(T, 2), so, bf(T // 2), ws)
+    with pytest.raises(ValueError, match="x_scale: required"):
+        mr.moe_layer(p, torch.zeros(n, 8), q(n), None, None, None, out, ws)
+    p.close()
+
+    p = mr.Plan(64, 256, 8, 2, 2, "bf16", "bf16", "bf16", inter=128)
+    T = p.recv_rows(n)
+    ws = torch.zeros(p.workspace_bytes, dtype=torch.uint8)
+    counts = torch.zeros(8, dtype=torch.int32)
+    off = torch.zeros(9, dtype=torch.int32)
+    wgu = torch.zeros(8, 256, 256, dtype=torch.bfloat16)
+    wd = torch.zeros(8, 256, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="h: shape"):
+        mr.moe_expert_swiglu(p, n, bf(T), counts, off, wgu, wd, bf(T, 64), bf(T), ws)
+    with pytest.raises(ValueError, match="w_down: shape"):
+        mr.moe_expert_swiglu(p, n, bf(T), counts, off, wgu, wd[:, :, :64], bf(T, 128), bf(T), ws)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        mr.moe_expert_swiglu(p, n, bf(T), counts, off, wgu, wd, bf(T, 128), bf(T), ws)
+    with pytest.raises(ValueError, match="w_gate_up: required"):
+        mr.moe_layer(p, torch.zeros(n, 8), bf(n), None, None, wd, out,
+                     torch.zeros(p.layer_workspace_bytes, dtype=torch.uint8))
+    p.close()
