@@ -55,6 +55,10 @@ def _sigs():
         "oracle_bf16_to_double": (ctypes.c_double, [ctypes.c_uint16]),
         "oracle_bf16_from_double": (ctypes.c_uint16, [ctypes.c_double]),
         "oracle_e4m3_to_double": (ctypes.c_double, [ctypes.c_uint8]),
+        "oracle_e4m3_from_float": (ctypes.c_uint8, [ctypes.c_float]),
+        "oracle_quant_rows": (ci, [i64, P, i32, i32, P, P, P]),
+        "oracle_fp8_gate_up_rows": (ci, [i64, P, P, i32, i32, i32, P, P, P, P, P, P, P]),
+        "oracle_fp8_down_rows": (ci, [i64, P, P, i32, i32, i32, P, P, P, P, P]),
     }
 
 
@@ -174,6 +178,64 @@ class Oracle:
                "swiglu")
         return (y, h) if want_h else y
 
+    def e4m3_from_float(self, v: float) -> int:
+        """Nearest finite e4m3 code, ties to even, saturating at +-448."""
+        return int(self.lib.oracle_e4m3_from_float(float(v)))
+
+    def quant_rows(self, rows: np.ndarray, h: np.ndarray, block: int):
+        """FP8 codes and per-block fp32 scales of the listed bf16 rows."""
+        rows = np.ascontiguousarray(rows, dtype=np.int32)
+        h = np.ascontiguousarray(h, dtype=np.uint16)
+        total, width = h.shape
+        q = np.zeros((total, width), np.uint8)
+        scale = np.zeros((total, width // block), np.float32)
+        _check(self.lib.oracle_quant_rows(rows.size, _p(rows), width, block, _p(h), _p(q),
+                                          _p(scale)), "quant")
+        return q, scale
+
+    def fp8_gate_up_rows(self, rows: np.ndarray, row_expert: np.ndarray, xq: np.ndarray,
+                         xs: np.ndarray, w_gate_up: np.ndarray, w_gate_up_scale: np.ndarray,
+                         block: int = 128, want_gu: bool = False):
+        """FP8 GEMM1 + SwiGLU on the listed rows: H bf16 bits (and g, u in double)."""
+        rows = np.ascontiguousarray(rows, dtype=np.int32)
+        row_expert = np.ascontiguousarray(row_expert, dtype=np.int32)
+        xq = np.ascontiguousarray(xq, dtype=np.uint8)
+        xs = np.ascontiguousarray(xs, dtype=np.float32)
+        w_gate_up = np.ascontiguousarray(w_gate_up, dtype=np.uint8)
+        w_gate_up_scale = np.ascontiguousarray(w_gate_up_scale, dtype=np.float32)
+        total, hidden = xq.shape
+        inter = w_gate_up.shape[1] // 2
+        assert w_gate_up.shape[2] == hidden and xs.shape == (total, hidden // block)
+        assert w_gate_up_scale.shape == (w_gate_up.shape[0], 2 * inter // block, hidden // block)
+        h = np.zeros((total, inter), np.uint16)
+        g = np.zeros((total, inter)) if want_gu else None
+        u = np.zeros((total, inter)) if want_gu else None
+        _check(self.lib.oracle_fp8_gate_up_rows(rows.size, _p(rows), _p(row_expert), hidden,
+                                                inter, block, _p(xq), _p(xs), _p(w_gate_up),
+                                                _p(w_gate_up_scale), _p(h), _p(g), _p(u)),
+               "fp8_gate_up")
+        return (h, g, u) if want_gu else h
+
+    def fp8_down_rows(self, rows: np.ndarray, row_expert: np.ndarray, hq: np.ndarray,
+                      hs: np.ndarray, w_down: np.ndarray, w_down_scale: np.ndarray,
+                      block: int = 128) -> np.ndarray:
+        """FP8 GEMM2 on the listed rows: Y bf16 bits."""
+        rows = np.ascontiguousarray(rows, dtype=np.int32)
+        row_expert = np.ascontiguousarray(row_expert, dtype=np.int32)
+        hq = np.ascontiguousarray(hq, dtype=np.uint8)
+        hs = np.ascontiguousarray(hs, dtype=np.float32)
+        w_down = np.ascontiguousarray(w_down, dtype=np.uint8)
+        w_down_scale = np.ascontiguousarray(w_down_scale, dtype=np.float32)
+        total, inter = hq.shape
+        hidden = w_down.shape[1]
+        assert w_down.shape[2] == inter and hs.shape == (total, inter // block)
+        assert w_down_scale.shape == (w_down.shape[0], hidden // block, inter // block)
+        y = np.zeros((total, hidden), np.uint16)
+        _check(self.lib.oracle_fp8_down_rows(rows.size, _p(rows), _p(row_expert), hidden, inter,
+                                             block, _p(hq), _p(hs), _p(w_down),
+                                             _p(w_down_scale), _p(y)), "fp8_down")
+        return y
+
     def combine(self, y: np.ndarray, y_dtype: str, topk_w: np.ndarray, slot_of: np.ndarray,
                 out_dtype: str) -> np.ndarray:
         y = np.ascontiguousarray(y, dtype=DT_NP[y_dtype])
@@ -235,7 +297,16 @@ class Oracle:
         res["recv"] = recv
         if inp.get("x_scale") is not None:
             res["recv_scale"] = self.scatter_rows(inp["x_scale"], slot_of, total)
-        if cfg.inter > 0:
+        if cfg.inter > 0 and cfg.x_dtype == "fp8_e4m3":
+            blk = cfg.scale_block
+            h = self.fp8_gate_up_rows(filled, idx.reshape(-1), recv, res["recv_scale"],
+                                      inp["w_gate_up"], inp["w_gate_up_scale"], blk)
+            hq, hs = self.quant_rows(filled, h, blk)
+            y = self.fp8_down_rows(filled, idx.reshape(-1), hq, hs, inp["w_down"],
+                                   inp["w_down_scale"], blk)
+            res["h"], res["hq"], res["h_scale"] = h, hq, hs
+            y_dtype = "bf16"
+        elif cfg.inter > 0:
             y = self.swiglu_rows(filled, idx.reshape(-1), recv, inp["w_gate_up"], inp["w_down"])
             y_dtype = "bf16"
         elif cfg.x_dtype == "fp8_e4m3":

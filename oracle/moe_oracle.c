@@ -32,6 +32,13 @@
  *             dispatch_local / dispatch_scatter_remote data-movement kernels).
  *   expert    identity (FP8 rows dequantised to bf16: code * block scale) or
  *             SwiGLU: H = bf16(silu(x Wg^T) * (x Wu^T)), Y = bf16(H Wd^T).
+ *             With FP8 rows the SwiGLU experts are FP8 too, reading the
+ *             dispatched codes and scales in place (the interface is agnostic
+ *             to the activation quantisation format, arXiv 2611.13188
+ *             abstract; the pages fix no FP8 GEMM format, so the readings
+ *             are: weights in e4m3 with one fp32 scale per 128x128 block, the
+ *             same 128-column granularity as the rows, and H quantised to
+ *             e4m3 per row and 128 columns by the rows' own amax / 448 rule).
  *   combine   out[t] = sum_j w[t,j] * Y[slot(t,j)] (Facts of PR 3158:
  *             combine_gather_remote and combine_weighted_sum).
  *
@@ -270,6 +277,131 @@ int oracle_swiglu_rows(int64_t n_rows, const int32_t* rows, const int32_t* row_e
         for (int32_t c = 0; c < hidden; ++c) {
             double acc = 0.0;
             for (int32_t d = 0; d < inter; ++d) acc += hbuf[d] * bf16_to_double(wd[(int64_t)c * inter + d]);
+            y[s * hidden + c] = bf16_from_double(acc);
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* ---------------------------------------------------------------- FP8 experts */
+
+/* Nearest finite e4m3 value to v, ties to the code whose last mantissa bit is
+ * 0, magnitudes of 448 and above giving +-448 (saturation instead of NaN;
+ * stated as a rule because distances to huge values round to ties).  Below
+ * 448, found by scanning the 127 non-negative finite codes in increasing
+ * order, where neighbouring codes are neighbouring values.  NaN inputs are
+ * outside the contract. */
+static uint8_t e4m3_from_float_satfinite(float v) {
+    double a = fabs((double)v);
+    uint8_t sign = signbit(v) ? 0x80 : 0;
+    if (a >= 448.0) return sign | 0x7E;
+    int best = 0;
+    double best_d = a;
+    for (int c = 1; c <= 0x7E; ++c) {
+        double d = fabs(e4m3_to_double((uint8_t)c) - a);
+        if (d < best_d || (d == best_d && (c & 1) == 0 && (best & 1) == 1)) {
+            best = c;
+            best_d = d;
+        }
+    }
+    return sign | (uint8_t)best;
+}
+
+uint8_t oracle_e4m3_from_float(float v) { return e4m3_from_float_satfinite(v); }
+
+/* FP8 quantisation of the listed bf16 rows, one fp32 scale per `block`
+ * columns: s = amax / 448 (1 for an all-zero block), code = e4m3(h / s).
+ * Both quotients are fp32 values: each is computed in double and rounded once
+ * to float, which is the correctly rounded fp32 quotient because double
+ * carries more than twice float's precision plus two bits (Figueroa, "When is
+ * double rounding innocuous?", 1995). */
+int oracle_quant_rows(int64_t n_rows, const int32_t* rows, int32_t width, int32_t block,
+                      const uint16_t* h, uint8_t* q, float* scale) {
+    if (block <= 0 || width % block) return ORACLE_BAD_ARG;
+    int32_t n_blocks = width / block;
+    for (int64_t i = 0; i < n_rows; ++i) {
+        int64_t s = rows[i];
+        for (int32_t b = 0; b < n_blocks; ++b) {
+            const uint16_t* hb = h + s * width + (int64_t)b * block;
+            double amax = 0.0;
+            for (int32_t c = 0; c < block; ++c) {
+                double a = fabs(bf16_to_double(hb[c]));
+                if (a > amax) amax = a;
+            }
+            float sc = amax > 0.0 ? (float)(amax / 448.0) : 1.0f;
+            scale[s * n_blocks + b] = sc;
+            for (int32_t c = 0; c < block; ++c) {
+                float v = (float)(bf16_to_double(hb[c]) / (double)sc);
+                q[s * width + (int64_t)b * block + c] = e4m3_from_float_satfinite(v);
+            }
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* FP8 SwiGLU gate/up step on the listed rows of the e4m3 buffer X (scales xs,
+ * one per row and `block` columns), row s using expert row_expert[i], whose
+ * e4m3 weights w_gate_up[e] (rows [0, I) gate, [I, 2I) up) carry one scale
+ * per block x block tile, ws[e][row / block][col / block]:
+ *   g[c] = sum_d (X[s,d] xs[s,d/block]) (Wg[c,d] ws[e][c/block][d/block])
+ *   u[c] = the same with row I + c,       h[c] = bf16(silu(g[c]) u[c])
+ * summed in double.  g_out, u_out (double [T, I]) may be NULL. */
+int oracle_fp8_gate_up_rows(int64_t n_rows, const int32_t* rows, const int32_t* row_expert,
+                            int32_t hidden, int32_t inter, int32_t block, const uint8_t* xq,
+                            const float* xs, const uint8_t* w_gate_up, const float* w_gate_up_s,
+                            uint16_t* h_out, double* g_out, double* u_out) {
+    if (block <= 0 || hidden % block || inter % block) return ORACLE_BAD_ARG;
+    int32_t kb = hidden / block;               /* scale blocks along the reduction */
+    int32_t rb = 2 * inter / block;            /* scale blocks along an expert's rows */
+    for (int64_t i = 0; i < n_rows; ++i) {
+        int64_t s = rows[i];
+        int64_t e = row_expert[i];
+        const uint8_t* xr = xq + s * hidden;
+        const float* xsr = xs + s * kb;
+        const uint8_t* w = w_gate_up + e * 2 * (int64_t)inter * hidden;
+        const float* wsc = w_gate_up_s + e * (int64_t)rb * kb;
+        for (int32_t c = 0; c < inter; ++c) {
+            int64_t cu = (int64_t)inter + c;
+            double g = 0.0, u = 0.0;
+            for (int32_t d = 0; d < hidden; ++d) {
+                double xv = e4m3_to_double(xr[d]) * (double)xsr[d / block];
+                g += xv * (e4m3_to_double(w[(int64_t)c * hidden + d]) *
+                           (double)wsc[(int64_t)(c / block) * kb + d / block]);
+                u += xv * (e4m3_to_double(w[cu * hidden + d]) *
+                           (double)wsc[(cu / block) * kb + d / block]);
+            }
+            if (g_out) g_out[s * inter + c] = g;
+            if (u_out) u_out[s * inter + c] = u;
+            h_out[s * inter + c] = bf16_from_double(g / (1.0 + exp(-g)) * u);
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* FP8 down projection on the listed rows of the e4m3 buffer H (scales hs, one
+ * per row and `block` columns), with expert e's e4m3 w_down[e] [D, I] and its
+ * per-tile scales wds[e][row / block][col / block]:
+ *   y[c] = bf16( sum_d (H[s,d] hs[s,d/block]) (Wd[c,d] wds[e][c/block][d/block]) ). */
+int oracle_fp8_down_rows(int64_t n_rows, const int32_t* rows, const int32_t* row_expert,
+                         int32_t hidden, int32_t inter, int32_t block, const uint8_t* hq,
+                         const float* hs, const uint8_t* w_down, const float* w_down_s,
+                         uint16_t* y) {
+    if (block <= 0 || hidden % block || inter % block) return ORACLE_BAD_ARG;
+    int32_t kb = inter / block;
+    int32_t rb = hidden / block;
+    for (int64_t i = 0; i < n_rows; ++i) {
+        int64_t s = rows[i];
+        int64_t e = row_expert[i];
+        const uint8_t* hr = hq + s * inter;
+        const float* hsr = hs + s * kb;
+        const uint8_t* w = w_down + e * (int64_t)hidden * inter;
+        const float* wsc = w_down_s + e * (int64_t)rb * kb;
+        for (int32_t c = 0; c < hidden; ++c) {
+            double acc = 0.0;
+            for (int32_t d = 0; d < inter; ++d)
+                acc += (e4m3_to_double(hr[d]) * (double)hsr[d / block]) *
+                       (e4m3_to_double(w[(int64_t)c * inter + d]) *
+                        (double)wsc[(int64_t)(c / block) * kb + d / block]);
             y[s * hidden + c] = bf16_from_double(acc);
         }
     }

@@ -271,6 +271,134 @@ def pin_swiglu_dense(o):
     assert np.all(_bf16_val(yz) == 0)
 
 
+# ------------------------------------------------------------------ FP8 experts
+def _e4m3_val(q: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(np.ascontiguousarray(q)).view(torch.float8_e4m3fn).double().numpy()
+
+
+def _fp8_codes(r, shape):
+    q = r.integers(0, 256, size=shape, dtype=np.uint8)
+    q[(q & 0x7F) == 0x7F] = 0x3C            # no NaN codes
+    return q
+
+
+def _distinct_pow2(r, shape, lo):
+    """Scales that are distinct powers of two, so that any mix-up of two
+    blocks' scales changes a result."""
+    count = int(np.prod(shape))
+    return (2.0 ** (lo - r.permutation(count))).reshape(shape).astype(np.float32)
+
+
+def pin_e4m3_encode(o):
+    """fp32 -> e4m3, nearest with ties to even and saturation at +-448: hand
+    cases (ties, subnormals, signed zero, overflow) and torch's
+    float8_e4m3fn cast (library) on random values inside the finite range."""
+    cases = [(1.0, 0x38), (1.0625, 0x38), (1.1875, 0x3A), (-1.75, 0xBE), (448.0, 0x7E),
+             (464.0, 0x7E), (500.0, 0x7E), (1e30, 0x7E), (-500.0, 0xFE), (2.0 ** -9, 0x01),
+             (2.0 ** -10, 0x00), (3 * 2.0 ** -10, 0x02), (0.0, 0x00), (-0.0, 0x80),
+             (2.0 ** -6, 0x08), (0.875 * 2.0 ** -6, 0x07)]
+    for v, code in cases:
+        assert o.e4m3_from_float(v) == code, (v, hex(o.e4m3_from_float(v)), hex(code))
+    r = _rng(10)
+    f = np.concatenate([r.uniform(-448, 448, 3000),
+                        r.choice([-1, 1], 3000) * 2.0 ** r.uniform(-12, 8.8, 3000)])
+    f = f.astype(np.float32)
+    ref = torch.from_numpy(f).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([o.e4m3_from_float(float(v)) for v in f], np.uint8)
+    assert np.array_equal(got, ref)
+
+
+def pin_quant_rows(o):
+    """H quantisation: the scale is the fp32 quotient amax / 448 (numpy
+    float32 division, IEEE), the codes are torch's e4m3 cast of the fp32
+    quotients h / scale; an all-zero block gets scale 1 and zero codes; rows
+    not listed stay untouched."""
+    r = _rng(11)
+    t, w, blk = 5, 384, 128
+    h = _bf16_bits(r.standard_normal((t, w)) * 10.0 ** r.integers(-3, 3, (t, 1)))
+    h[2, 128:256] = 0
+    h[3, :128] = _bf16_bits(np.linspace(-448, 448, 128))     # amax 448: scale 1
+    rows = np.arange(t, dtype=np.int32)
+    q, sc = o.quant_rows(rows, h, blk)
+    hv = _bf16_val(h).astype(np.float32)                       # exact: bf16 is a subset
+    amax = np.abs(hv).reshape(t, w // blk, blk).max(axis=2)
+    sc_ref = np.where(amax > 0, amax / np.float32(448), np.float32(1)).astype(np.float32)
+    assert np.array_equal(sc, sc_ref)
+    assert sc[2, 1] == 1.0 and np.all(q[2, 128:256] == 0) and sc[3, 0] == 1.0
+    quo = (hv.reshape(t, w // blk, blk) / sc_ref[:, :, None]).astype(np.float32).reshape(t, w)
+    ref = torch.from_numpy(np.clip(quo, -448, 448)).to(torch.float8_e4m3fn).view(torch.uint8)
+    assert np.array_equal(q, ref.numpy())
+    q1, sc1 = o.quant_rows(np.array([4], np.int32), h, blk)
+    assert np.all(q1[:4] == 0) and np.all(sc1[:4] == 0) and np.array_equal(q1[4], q[4])
+
+
+def pin_fp8_gate_up_dense(o):
+    """FP8 GEMM1 + SwiGLU against numpy float64 matmuls (library) of operands
+    dequantised here, the weight scale grid expanded with np.kron: g and u
+    agree to double rounding, h = bf16(silu(g) u) to half a bf16 ulp.  The
+    scales are distinct powers of two, so a wrong block index, a dropped
+    scale or the gate's scale on the up rows fails."""
+    r = _rng(12)
+    rows_n, d, inter, e, blk = 5, 256, 256, 2, 128
+    xq = _fp8_codes(r, (rows_n, d))
+    xs = _distinct_pow2(r, (rows_n, d // blk), -2)
+    wq = _fp8_codes(r, (e, 2 * inter, d))
+    ws = _distinct_pow2(r, (e, 2 * inter // blk, d // blk), -4)
+    rows = np.arange(rows_n, dtype=np.int32)
+    xv = _e4m3_val(xq) * np.repeat(xs.astype(np.float64), blk, axis=1)
+    for ex in range(e):
+        h, g, u = o.fp8_gate_up_rows(rows, np.full(rows_n, ex, np.int32), xq, xs, wq, ws, blk,
+                                     want_gu=True)
+        wv = _e4m3_val(wq[ex]) * np.kron(ws[ex].astype(np.float64), np.ones((blk, blk)))
+        g_ref, u_ref = xv @ wv[:inter].T, xv @ wv[inter:].T
+        g_abs, u_abs = np.abs(xv) @ np.abs(wv[:inter]).T, np.abs(xv) @ np.abs(wv[inter:]).T
+        assert np.all(np.abs(g - g_ref) <= 1e-12 * g_abs)
+        assert np.all(np.abs(u - u_ref) <= 1e-12 * u_abs)
+        with np.errstate(over="ignore"):
+            h_ref = g / (1.0 + np.exp(-g)) * u
+        # half a bf16 ulp: 2^-8 relative, or half the subnormal quantum 2^-133
+        assert np.all(np.abs(_bf16_val(h) - h_ref) <= np.abs(h_ref) * 2 ** -8 + 2.0 ** -134)
+
+
+def pin_fp8_down_dense(o):
+    """FP8 GEMM2 against a numpy float64 matmul (library) of operands
+    dequantised here (row scales by np.repeat, weight tiles by np.kron), with
+    distinct power-of-two scales; y within half a bf16 ulp; the expert id
+    selects the weights."""
+    r = _rng(13)
+    rows_n, d, inter, e, blk = 6, 256, 384, 3, 128
+    hq = _fp8_codes(r, (rows_n, inter))
+    hs = _distinct_pow2(r, (rows_n, inter // blk), 0)
+    wq = _fp8_codes(r, (e, d, inter))
+    ws = _distinct_pow2(r, (e, d // blk, inter // blk), -6)
+    rows = np.arange(rows_n, dtype=np.int32)
+    re = (np.arange(rows_n) % e).astype(np.int32)
+    y = o.fp8_down_rows(rows, re, hq, hs, wq, ws, blk)
+    hv = _e4m3_val(hq) * np.repeat(hs.astype(np.float64), blk, axis=1)
+    for i in range(rows_n):
+        wv = _e4m3_val(wq[re[i]]) * np.kron(ws[re[i]].astype(np.float64), np.ones((blk, blk)))
+        y_ref = wv @ hv[i]
+        assert np.all(np.abs(_bf16_val(y[i]) - y_ref) <= np.abs(y_ref) * 2 ** -8 + 2.0 ** -134)
+
+
+def pin_fp8_gate_up_equals_bf16_with_unit_scales(o):
+    """With every scale 1 the FP8 gate/up step is the (separately pinned) bf16
+    SwiGLU step on the decoded values, bit for bit: every e4m3 value is a bf16
+    value, and both sum the same products in the same order."""
+    r = _rng(14)
+    rows_n, d, inter, blk = 4, 256, 128, 128
+    xq = _fp8_codes(r, (rows_n, d))
+    wq = _fp8_codes(r, (1, 2 * inter, d))
+    rows = np.arange(rows_n, dtype=np.int32)
+    ex = np.zeros(rows_n, np.int32)
+    h8 = o.fp8_gate_up_rows(rows, ex, xq, np.ones((rows_n, d // blk), np.float32), wq,
+                            np.ones((1, 2 * inter // blk, d // blk), np.float32), blk)
+    as_bf16 = lambda q: _bf16_bits(_e4m3_val(q))  # noqa: E731  (exact)
+    _, h16 = o.swiglu_rows(rows, ex, as_bf16(xq), as_bf16(wq), np.zeros((1, d, inter), np.uint16),
+                           want_h=True)
+    assert np.array_equal(h8, h16)
+
+
 # ------------------------------------------------------------------ combine
 def pin_combine_identity_roundtrip(o):
     """combine(dispatch(x)) with identity experts and renormalised weights is

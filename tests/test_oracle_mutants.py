@@ -25,7 +25,9 @@ MUTANTS = {
                                "            uint16_t hb = bf16_from_double(silu * u);",
                                "double silu = u / (1.0 + exp(-u));\n"
                                "            uint16_t hb = bf16_from_double(silu * g);"),
-    "silu_sign": ("g / (1.0 + exp(-g))", "g / (1.0 + exp(g))"),
+    "silu_sign": ("double silu = g / (1.0 + exp(-g));", "double silu = g / (1.0 + exp(g));"),
+    "fp8_silu_sign": ("bf16_from_double(g / (1.0 + exp(-g)) * u)",
+                      "bf16_from_double(g / (1.0 + exp(g)) * u)"),
     "w_down_transposed": ("wd[(int64_t)c * inter + d]", "wd[(int64_t)d * hidden + c]"),
     "combine_weight_index": ("acc += (double)topk_w[t * top_k + j] * load_elem",
                              "acc += (double)topk_w[t * top_k] * load_elem"),
@@ -44,6 +46,22 @@ MUTANTS = {
     "e4m3_bias": ("ldexp(1.0 + (double)m / 8.0, ex - 7)", "ldexp(1.0 + (double)m / 8.0, ex - 8)"),
     "e4m3_subnormal": ("ldexp((double)m / 8.0, -6)", "ldexp((double)m / 8.0, -7)"),
     "bf16_decode_shift": ("(uint32_t)b << 16", "(uint32_t)b << 15"),
+    "e4m3_encode_ties_odd": ("(c & 1) == 0 && (best & 1) == 1", "(c & 1) == 1 && (best & 1) == 0"),
+    "e4m3_encode_no_saturation": ("if (a >= 448.0) return sign | 0x7E;", ""),
+    "quant_divisor": ("(float)(amax / 448.0)", "(float)(amax / 240.0)"),
+    "quant_signed_amax": ("double a = fabs(bf16_to_double(hb[c]));",
+                          "double a = bf16_to_double(hb[c]);"),
+    "fp8_x_scale_dropped": ("double xv = e4m3_to_double(xr[d]) * (double)xsr[d / block];",
+                            "double xv = e4m3_to_double(xr[d]);"),
+    "fp8_gate_scale_transposed": ("(double)wsc[(int64_t)(c / block) * kb + d / block]);\n"
+                                  "                u +=",
+                                  "(double)wsc[(int64_t)(d / block) * kb + c / block]);\n"
+                                  "                u +="),
+    "fp8_up_uses_gate_scale": ("(double)wsc[(cu / block) * kb + d / block]",
+                               "(double)wsc[(int64_t)(c / block) * kb + d / block]"),
+    "fp8_down_h_scale_block": ("(double)hsr[d / block]", "(double)hsr[0]"),
+    "fp8_down_expert_scales": ("const float* wsc = w_down_s + e * (int64_t)rb * kb;",
+                               "const float* wsc = w_down_s;"),
 }
 
 

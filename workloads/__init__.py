@@ -14,7 +14,9 @@ in the order logits, x, expert weights.
 FP8 inputs: each 128-column block of a row gets ``scale = amax / 448`` (1 when
 the block is all zero), the block is divided by its scale, clamped to the
 e4m3 finite range and rounded to nearest-even by torch's float8_e4m3fn cast.
-That is input preparation: the method receives the FP8 codes and the scales.
+With FP8 rows the SwiGLU expert weights are FP8 as well, quantised the same
+way per 128x128 tile.  That is input preparation: the method receives the FP8
+codes and the scales.
 """
 from __future__ import annotations
 
@@ -64,6 +66,10 @@ CONFIGS = {
     "skewed": Config("skewed", 16384, 4096, 128, 4, 4, logits="zipf1.2"),
     # N=1024, D=7168, bf16, E=64, k=8, SwiGLU experts with I=2048.
     "layer": Config("layer", 1024, 7168, 64, 8, 8, inter=2048),
+    # The same layer with FP8 rows (per-128-column scales, as dispatched at
+    # prefill) and FP8 expert weights (one scale per 128x128 tile).
+    "layer_fp8": Config("layer_fp8", 1024, 7168, 64, 8, 8, "fp8_e4m3", "bf16", "bf16",
+                        scale_block=128, inter=2048),
 }
 
 
@@ -86,6 +92,17 @@ def _quantise_fp8_blocks(xf: torch.Tensor, block: int):
     return q.contiguous(), scale.to(torch.float32).contiguous()
 
 
+def _quantise_fp8_tiles(wf: torch.Tensor, block: int):
+    """Per-(block x block tile) amax scaling of a weight matrix to e4m3 codes."""
+    r, c = wf.shape
+    wb = wf.view(r // block, block, c // block, block)
+    amax = wb.abs().amax(dim=(1, 3))
+    scale = torch.where(amax > 0, amax / FP8_E4M3_MAX, torch.ones_like(amax))
+    q = (wb / scale[:, None, :, None]).clamp(-FP8_E4M3_MAX, FP8_E4M3_MAX)
+    q = q.to(torch.float8_e4m3fn).view(r, c).view(torch.uint8)
+    return q.contiguous(), scale.to(torch.float32).contiguous()
+
+
 def make_inputs(cfg: Config, seed: int = 0, n: int | None = None,
                 with_weights: bool | None = None) -> dict:
     """Draw one batch of inputs on the CPU.
@@ -96,6 +113,9 @@ def make_inputs(cfg: Config, seed: int = 0, n: int | None = None,
       x_scale [N, D/128] float32 or None
       w_gate_up [E, 2I, D] bfloat16 (gate rows first, then up rows) or None
       w_down    [E, D, I]  bfloat16 or None
+    With FP8 rows the weights are e4m3 codes (uint8) instead, with
+      w_gate_up_scale [E, 2I/128, D/128] and w_down_scale [E, D/128, I/128]
+    float32, one scale per 128x128 tile.
     """
     n = cfg.n if n is None else n
     g = torch.Generator("cpu").manual_seed(seed)
@@ -115,10 +135,21 @@ def make_inputs(cfg: Config, seed: int = 0, n: int | None = None,
     else:
         raise ValueError(cfg.x_dtype)
     out = {"logits": logits.contiguous(), "x": x.contiguous(), "x_scale": x_scale,
-           "w_gate_up": None, "w_down": None}
+           "w_gate_up": None, "w_down": None, "w_gate_up_scale": None, "w_down_scale": None}
     if with_weights is None:
         with_weights = cfg.inter > 0
-    if with_weights:
+    if with_weights and cfg.x_dtype == "fp8_e4m3":
+        e, d, i, b = cfg.n_experts, cfg.hidden, cfg.inter, cfg.scale_block
+        wgu = torch.empty(e, 2 * i, d, dtype=torch.uint8)
+        wd = torch.empty(e, d, i, dtype=torch.uint8)
+        sgu = torch.empty(e, 2 * i // b, d // b, dtype=torch.float32)
+        sd = torch.empty(e, d // b, i // b, dtype=torch.float32)
+        for ex in range(e):
+            wgu[ex], sgu[ex] = _quantise_fp8_tiles(torch.randn(2 * i, d, generator=g) * cfg.w_std, b)
+        for ex in range(e):
+            wd[ex], sd[ex] = _quantise_fp8_tiles(torch.randn(d, i, generator=g) * cfg.w_std, b)
+        out.update(w_gate_up=wgu, w_down=wd, w_gate_up_scale=sgu, w_down_scale=sd)
+    elif with_weights:
         e, d, i = cfg.n_experts, cfg.hidden, cfg.inter
         wgu = torch.empty(e, 2 * i, d, dtype=torch.bfloat16)
         wd = torch.empty(e, d, i, dtype=torch.bfloat16)
