@@ -15,7 +15,8 @@ import torch
 
 __all__ = [
     "MoeError", "Plan", "LIB_PATH", "moe_route_topk", "moe_dispatch", "moe_route_dispatch",
-    "moe_expert_dequant", "moe_expert_swiglu", "moe_combine", "moe_layer", "moe_layer_buffer",
+    "moe_expert_dequant", "moe_expert_swiglu", "moe_expert_swiglu_fp8", "moe_combine",
+    "moe_layer", "moe_layer_fp8", "moe_layer_buffer",
     "moe_get_status", "moe_workspace_init", "moe_strerror", "DTYPE_CODES", "ELEM_BYTES",
     "FUSED_MAX_TOKENS",
 ]
@@ -56,8 +57,10 @@ _SIGS = {
     "moe_route_dispatch": (ctypes.c_int, [_P, _i32] + [_P] * 13),
     "moe_expert_dequant": (ctypes.c_int, [_P, _i32, _P, _P, _P, _P, _P, _P]),
     "moe_expert_swiglu": (ctypes.c_int, [_P, _i32, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_expert_swiglu_fp8": (ctypes.c_int, [_P, _i32] + [_P] * 15),
     "moe_combine": (ctypes.c_int, [_P, _i32, _P, _P, _P, _P, _P, _P]),
     "moe_layer": (ctypes.c_int, [_P, _i32, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_layer_fp8": (ctypes.c_int, [_P, _i32] + [_P] * 10),
     "moe_layer_buffer": (_P, [_P, _P, ctypes.c_char_p]),
     "moe_get_status": (ctypes.c_int, [_P, _P, _P]),
     "moe_workspace_init": (ctypes.c_int, [_P, _P, _P]),
@@ -221,7 +224,15 @@ class Plan:
             b["y"] = torch.empty(T, D, dtype=_TORCH[self.y_dtype][0], device=device)
         if self.inter > 0:
             b["h"] = torch.empty(T, self.inter, dtype=torch.bfloat16, device=device)
+        if self.fp8_experts:
+            b["hq"] = torch.empty(T, self.inter, dtype=torch.uint8, device=device)
+            b["h_scale"] = torch.empty(T, self.inter // 128, dtype=torch.float32, device=device)
         return b
+
+    @property
+    def fp8_experts(self) -> bool:
+        """SwiGLU experts on FP8 rows run in FP8 (moe_expert_swiglu_fp8)."""
+        return self.inter > 0 and self.x_dtype == "fp8_e4m3"
 
 
 def moe_route_topk(plan: Plan, logits, topk_idx, topk_w, counts, expert_off, ws, stream=None):
@@ -303,6 +314,38 @@ def moe_expert_swiglu(plan: Plan, n: int, recv, counts, expert_off, w_gate_up, w
                                   _stream(stream)), "moe_expert_swiglu")
 
 
+def _expect_fp8_weights(plan: Plan, w_gate_up, w_gate_up_scale, w_down, w_down_scale):
+    E, D, I = plan.n_experts, plan.hidden, plan.inter
+    _expect(w_gate_up, _TORCH["fp8_e4m3"], (E, 2 * I, D), "w_gate_up")
+    _expect(w_gate_up_scale, (torch.float32,), (E, 2 * I // 128, D // 128), "w_gate_up_scale")
+    _expect(w_down, _TORCH["fp8_e4m3"], (E, D, I), "w_down")
+    _expect(w_down_scale, (torch.float32,), (E, D // 128, I // 128), "w_down_scale")
+
+
+def moe_expert_swiglu_fp8(plan: Plan, n: int, recv, recv_scale, counts, expert_off, slot_of,
+                          w_gate_up, w_gate_up_scale, w_down, w_down_scale, h, hq, h_scale, y,
+                          ws, stream=None):
+    """FP8 SwiGLU experts on the FP8 receive buffer: GEMM1 -> H (bf16) ->
+    per-128-column e4m3 Hq and scales -> GEMM2 -> Y (bf16)."""
+    E, D, I = plan.n_experts, plan.hidden, plan.inter
+    T = plan.recv_rows(n)
+    _expect_fp8_weights(plan, w_gate_up, w_gate_up_scale, w_down, w_down_scale)
+    _expect_rows(recv, _TORCH["fp8_e4m3"], T, D, "recv")
+    _expect_rows(recv_scale, (torch.float32,), T, D // 128, "recv_scale")
+    _expect(counts, (torch.int32,), (E,), "counts")
+    _expect(expert_off, (torch.int32,), (E + 1,), "expert_off")
+    _expect(slot_of, (torch.int32,), (n, plan.top_k), "slot_of")
+    _expect_rows(h, (torch.bfloat16,), T, I, "h")
+    _expect_rows(hq, _TORCH["fp8_e4m3"], T, I, "hq")
+    _expect_rows(h_scale, (torch.float32,), T, I // 128, "h_scale")
+    _expect_rows(y, (torch.bfloat16,), T, D, "y")
+    _check(_lib.moe_expert_swiglu_fp8(plan.handle, n, _ptr(recv), _ptr(recv_scale), _ptr(counts),
+                                      _ptr(expert_off), _ptr(slot_of), _ptr(w_gate_up),
+                                      _ptr(w_gate_up_scale), _ptr(w_down), _ptr(w_down_scale),
+                                      _ptr(h), _ptr(hq), _ptr(h_scale), _ptr(y), _ws(plan, ws),
+                                      _stream(stream)), "moe_expert_swiglu_fp8")
+
+
 def moe_combine(plan: Plan, y, topk_w, slot_of, out, ws, stream=None):
     n = out.shape[0]
     _expect(out, _TORCH[plan.out_dtype], (n, plan.hidden), "out")
@@ -319,13 +362,29 @@ def moe_layer(plan: Plan, logits, x, x_scale, w_gate_up, w_down, out, ws, stream
     _expect(x, _TORCH[plan.x_dtype], (n, plan.hidden), "x")
     _expect(out, _TORCH[plan.out_dtype], (n, plan.hidden), "out")
     _expect_scales(plan, x_scale, n, "x_scale", exact=True)
-    if plan.inter > 0:
+    if plan.inter > 0 and not plan.fp8_experts:
         E, D, I = plan.n_experts, plan.hidden, plan.inter
         _expect(w_gate_up, (torch.bfloat16,), (E, 2 * I, D), "w_gate_up")
         _expect(w_down, (torch.bfloat16,), (E, D, I), "w_down")
     _check(_lib.moe_layer(plan.handle, n, _ptr(logits), _ptr(x), _ptr(x_scale), _ptr(w_gate_up),
                           _ptr(w_down), _ptr(out), _ws(plan, ws, layer=True), _stream(stream)),
            "moe_layer")
+
+
+def moe_layer_fp8(plan: Plan, logits, x, x_scale, w_gate_up, w_gate_up_scale, w_down,
+                  w_down_scale, out, ws, stream=None):
+    """moe_layer for plans with FP8 experts (FP8 rows and inter > 0)."""
+    n = x.shape[0]
+    _expect(logits, (torch.float32,), (n, plan.n_experts), "logits")
+    _expect(x, _TORCH[plan.x_dtype], (n, plan.hidden), "x")
+    _expect(out, _TORCH[plan.out_dtype], (n, plan.hidden), "out")
+    _expect_scales(plan, x_scale, n, "x_scale", exact=True)
+    if plan.fp8_experts:
+        _expect_fp8_weights(plan, w_gate_up, w_gate_up_scale, w_down, w_down_scale)
+    _check(_lib.moe_layer_fp8(plan.handle, n, _ptr(logits), _ptr(x), _ptr(x_scale),
+                              _ptr(w_gate_up), _ptr(w_gate_up_scale), _ptr(w_down),
+                              _ptr(w_down_scale), _ptr(out), _ws(plan, ws, layer=True),
+                              _stream(stream)), "moe_layer_fp8")
 
 
 def moe_layer_buffer(plan: Plan, ws, name: str, dtype, shape) -> torch.Tensor:

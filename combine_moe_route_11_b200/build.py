@@ -20,6 +20,7 @@ LIB = os.path.join(PKG, "libmoeroute.so")
 OBJ_DIR = os.path.join(PKG, "_build")
 
 SOURCES = ["api.cu", "route.cu", "route_dispatch.cu", "dispatch.cu", "combine.cu", "swiglu_gemm.cu",
+           "fp8_gemm.cu",
            "route_noalloc.cu"]
 HEADERS = ["moe_internal.cuh", "route_common.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -1,7 +1,7 @@
 // C ABI of libmoeroute: plan validation, workspace layout and the entry
 // points declared in include/moeroute.h.  Host code only; every step of the
 // path runs in the kernels of route.cu, route_dispatch.cu, dispatch.cu,
-// combine.cu, swiglu_gemm.cu and route_noalloc.cu.  The per-device caches
+// combine.cu, swiglu_gemm.cu, fp8_gemm.cu and route_noalloc.cu.  The per-device caches
 // here and in the launchers may be reached from several host threads.
 #include "moe_internal.cuh"
 
@@ -84,8 +84,11 @@ Layout make_layout(const moe_plan& p) {
   L.recv = take(T * d.hidden * elem_bytes(d.x_dtype));
   L.recv_scale = take(T * p.scale_cols * 4);
   const bool needs_y = d.inter > 0 || d.x_dtype == MOE_FP8_E4M3;
+  const bool fp8_experts = d.inter > 0 && d.x_dtype == MOE_FP8_E4M3;
   L.y = take(needs_y ? T * d.hidden * elem_bytes(d.y_dtype) : 0);
   L.h = take(d.inter > 0 ? T * size_t(d.inter) * 2 : 0);
+  L.hq = take(fp8_experts ? T * size_t(d.inter) : 0);
+  L.h_scale = take(fp8_experts ? T * size_t(d.inter / 128) * 4 : 0);
   L.end = at;
   return L;
 }
@@ -132,7 +135,10 @@ moe_status moe_plan_create(const moe_desc* desc, moe_plan** out) {
   }
   if (d.inter < 0) return MOE_ERR_INVALID_ARG;
   if (d.inter > 0) {
-    if (d.x_dtype != MOE_BF16 || d.y_dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+    // bf16 experts on bf16 rows, or FP8 experts on FP8 rows with 128-column scales
+    const bool fp8 = d.x_dtype == MOE_FP8_E4M3;
+    if ((d.x_dtype != MOE_BF16 && !fp8) || d.y_dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+    if (fp8 && d.scale_block != 128) return MOE_ERR_UNSUPPORTED;
     if (d.hidden % 256 || d.inter % 128) return MOE_ERR_UNSUPPORTED;
   }
   moe_plan tmp;
@@ -231,7 +237,7 @@ moe_status moe_expert_swiglu(const moe_plan* p, int32_t n, const void* recv, con
                              void* h, void* y, void* ws, moe_stream_t stream) {
   moe_status s = check_call(p, n, ws);
   if (s != MOE_OK) return s;
-  if (p->d.inter <= 0) return MOE_ERR_UNSUPPORTED;
+  if (p->d.inter <= 0 || p->d.x_dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
   if (n == 0) return MOE_OK;
   if (!recv || !counts || !expert_off || !w_gate_up || !w_down || !h || !y)
     return MOE_ERR_INVALID_ARG;
@@ -240,6 +246,27 @@ moe_status moe_expert_swiglu(const moe_plan* p, int32_t n, const void* recv, con
     return MOE_ERR_INVALID_ARG;
   return cuda_status(launch_swiglu(*p, n, recv, counts, expert_off, w_gate_up, w_down, h, y, ws,
                                    reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_expert_swiglu_fp8(const moe_plan* p, int32_t n, const void* recv,
+                                 const float* recv_scale, const int32_t* counts,
+                                 const int32_t* expert_off, const int32_t* slot_of,
+                                 const void* w_gate_up, const float* w_gate_up_scale,
+                                 const void* w_down, const float* w_down_scale, void* h, void* hq,
+                                 float* h_scale, void* y, void* ws, moe_stream_t stream) {
+  moe_status s = check_call(p, n, ws);
+  if (s != MOE_OK) return s;
+  if (p->d.inter <= 0 || p->d.x_dtype != MOE_FP8_E4M3) return MOE_ERR_UNSUPPORTED;
+  if (n == 0) return MOE_OK;
+  if (!recv || !recv_scale || !counts || !expert_off || !slot_of || !w_gate_up ||
+      !w_gate_up_scale || !w_down || !w_down_scale || !h || !hq || !h_scale || !y)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(recv) || !aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(h) ||
+      !aligned16(hq) || !aligned16(y))
+    return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_swiglu_fp8(*p, n, recv, recv_scale, counts, expert_off, slot_of,
+                                       w_gate_up, w_gate_up_scale, w_down, w_down_scale, h, hq,
+                                       h_scale, y, ws, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_combine(const moe_plan* p, int32_t n, const void* y, const float* topk_w,
@@ -260,18 +287,28 @@ void* moe_layer_buffer(const moe_plan* p, void* ws, const char* name) {
   struct { const char* n; size_t off; } tab[] = {
       {"topk_idx", L.topk_idx}, {"topk_w", L.topk_w},   {"counts", L.counts},
       {"expert_off", L.expert_off}, {"slot_of", L.slot_of}, {"src_of", L.src_of},
-      {"recv", L.recv},         {"recv_scale", L.recv_scale}, {"y", L.y}, {"h", L.h}};
+      {"recv", L.recv},         {"recv_scale", L.recv_scale}, {"y", L.y}, {"h", L.h},
+      {"hq", L.hq},             {"h_scale", L.h_scale}};
   for (auto& e : tab)
     if (strcmp(e.n, name) == 0) return b + e.off;
   return nullptr;
 }
 
-moe_status moe_layer(const moe_plan* p, int32_t n, const float* logits, const void* x,
-                     const float* x_scale, const void* w_gate_up, const void* w_down, void* out,
-                     void* ws, moe_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// route -> dispatch -> expert -> combine on one stream; the weight scales are
+// those of FP8 experts (null for bf16 or identity experts).
+moe_status layer_impl(const moe_plan* p, int32_t n, const float* logits, const void* x,
+                      const float* x_scale, const void* w_gate_up, const float* w_gate_up_scale,
+                      const void* w_down, const float* w_down_scale, void* out, void* ws,
+                      moe_stream_t stream) {
   moe_status s = check_call(p, n, ws);
   if (s != MOE_OK) return s;
   const moe_desc& d = p->d;
+  const bool fp8_experts = d.inter > 0 && d.x_dtype == MOE_FP8_E4M3;
+  if (fp8_experts && (!w_gate_up_scale || !w_down_scale)) return MOE_ERR_INVALID_ARG;
   // Every argument error is found here, before the first launch: the stages
   // below only receive pointers into ws (256-byte aligned by the layout) or
   // arguments checked here, so none of them can reject the call halfway.
@@ -302,7 +339,12 @@ moe_status moe_layer(const moe_plan* p, int32_t n, const float* logits, const vo
                          recv_scale, slot_of, src_of, ws, stream);
   if (s != MOE_OK || n == 0) return s;
   const void* yin = recv;
-  if (d.inter > 0) {
+  if (fp8_experts) {
+    s = moe_expert_swiglu_fp8(p, n, recv, recv_scale, counts, expert_off, slot_of, w_gate_up,
+                              w_gate_up_scale, w_down, w_down_scale, h, b + L.hq,
+                              reinterpret_cast<float*>(b + L.h_scale), y, ws, stream);
+    yin = y;
+  } else if (d.inter > 0) {
     s = moe_expert_swiglu(p, n, recv, counts, expert_off, w_gate_up, w_down, h, y, ws, stream);
     yin = y;
   } else if (d.x_dtype == MOE_FP8_E4M3) {
@@ -311,6 +353,28 @@ moe_status moe_layer(const moe_plan* p, int32_t n, const float* logits, const vo
   }
   if (s != MOE_OK) return s;
   return moe_combine(p, n, yin, topk_w, slot_of, out, ws, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_layer(const moe_plan* p, int32_t n, const float* logits, const void* x,
+                     const float* x_scale, const void* w_gate_up, const void* w_down, void* out,
+                     void* ws, moe_stream_t stream) {
+  // FP8 experts need their weight scales: moe_layer_fp8
+  if (p && p->d.inter > 0 && p->d.x_dtype == MOE_FP8_E4M3) return MOE_ERR_UNSUPPORTED;
+  return layer_impl(p, n, logits, x, x_scale, w_gate_up, nullptr, w_down, nullptr, out, ws,
+                    stream);
+}
+
+moe_status moe_layer_fp8(const moe_plan* p, int32_t n, const float* logits, const void* x,
+                         const float* x_scale, const void* w_gate_up, const float* w_gate_up_scale,
+                         const void* w_down, const float* w_down_scale, void* out, void* ws,
+                         moe_stream_t stream) {
+  if (p && !(p->d.inter > 0 && p->d.x_dtype == MOE_FP8_E4M3)) return MOE_ERR_UNSUPPORTED;
+  return layer_impl(p, n, logits, x, x_scale, w_gate_up, w_gate_up_scale, w_down, w_down_scale,
+                    out, ws, stream);
 }
 
 moe_status moe_get_status(const moe_plan* p, void* ws, moe_stream_t stream) {

@@ -39,7 +39,9 @@ inline int elem_bytes(int dtype) {
 // Byte offsets of every buffer inside a workspace, fixed by n_max.
 struct Layout {
   size_t ctrl, totals, masks, blk, bases, rank, route_end;
-  size_t topk_idx, topk_w, counts, expert_off, slot_of, src_of, recv, recv_scale, y, h, end;
+  size_t topk_idx, topk_w, counts, expert_off, slot_of, src_of, recv, recv_scale, y, h;
+  size_t hq, h_scale;  // FP8 SwiGLU experts: H in e4m3 and its per-128-column scales
+  size_t end;
 };
 
 }  // namespace moe
@@ -93,6 +95,14 @@ cudaError_t launch_combine(const moe_plan& p, int32_t n, const void* y, const fl
 cudaError_t launch_swiglu(const moe_plan& p, int32_t n, const void* recv, const int32_t* counts,
                           const int32_t* expert_off, const void* w_gate_up, const void* w_down,
                           void* h, void* y, void* ws, cudaStream_t st);
+cudaError_t launch_swiglu_fp8(const moe_plan& p, int32_t n, const void* recv,
+                              const float* recv_scale, const int32_t* counts,
+                              const int32_t* expert_off, const int32_t* slot_of,
+                              const void* w_gate_up, const float* w_gate_up_scale,
+                              const void* w_down, const float* w_down_scale, void* h, void* hq,
+                              float* h_scale, void* y, void* ws, cudaStream_t st);
+// The driver's cuTensorMapEncodeTiled (null if unavailable), looked up once.
+void* tensor_map_encoder();
 
 // Launch with programmatic stream serialization: the kernel may be scheduled
 // while the previous kernel of the stream finishes, and must call

@@ -443,17 +443,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------- host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+}  // namespace
+
+void* tensor_map_encoder() {
   // looked up once (thread-safe static initialisation); null if unavailable
-  static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+  static void* const fn = [] {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
         q != cudaDriverEntryPointSuccess)
       p = nullptr;
-    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    return p;
   }();
   return fn;
+}
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encoder());
 }
 
 // 2D bf16 tensor map over a row-major [rows, cols] matrix; box = 64 columns

@@ -17,7 +17,9 @@
  *                    ("MLX expert parallelism all_to_all PR 3158", Facts:
  *                    dispatch_local / dispatch_scatter_remote).
  *   moe_route_dispatch  the two calls above as one launch for small batches.
- *   moe_expert_*     the expert step reading the dispatched buffer in place:
+ *   moe_expert_*     the expert step reading the dispatched buffer in place
+ *                    (bf16, or FP8 with its scales, the interface being
+ *                    agnostic to the activation quantisation format):
  *                    grouped GEMMs read the rank-major buffer instead of a
  *                    per-expert copy (arXiv 2611.13188 abstract); segments are
  *                    contiguous, which is the promise a sorted-index grouped
@@ -110,7 +112,8 @@ typedef struct moe_plan moe_plan;
 /* Validate `desc` and build a plan (host only, no CUDA call).
  * Requires: every row (x, Y, out) a multiple of 16 bytes; scale_block > 0
  * only with FP8 rows and dividing D; T(n_max) < 2^31; for inter > 0 also
- * x = y = BF16, D % 256 == 0 and I % 128 == 0.  *out is set only on MOE_OK. */
+ * y = BF16, D % 256 == 0, I % 128 == 0 and either x = BF16 (bf16 experts) or
+ * x = FP8 with scale_block = 128 (FP8 experts).  *out is set only on MOE_OK. */
 MOE_API moe_status moe_plan_create(const moe_desc* desc, moe_plan** out);
 MOE_API void moe_plan_destroy(moe_plan* plan);
 
@@ -183,11 +186,38 @@ MOE_API moe_status moe_expert_dequant(const moe_plan* plan, int32_t n, const voi
  * fp32 accumulation on the tensor cores.  w_gate_up: device bf16 [E, 2I, D]
  * (rows [0, I) are Wg[e], rows [I, 2I) are Wu[e]); w_down: device bf16
  * [E, D, I]; recv: device bf16 [T, D]; h: device bf16 [T, I]; y: device bf16
- * [T, D].  counts and expert_off as written by moe_route_topk. */
+ * [T, D].  counts and expert_off as written by moe_route_topk.  Plans with
+ * bf16 rows only (FP8 rows: moe_expert_swiglu_fp8). */
 MOE_API moe_status moe_expert_swiglu(const moe_plan* plan, int32_t n, const void* recv,
                              const int32_t* counts, const int32_t* expert_off,
                              const void* w_gate_up, const void* w_down, void* h, void* y,
                              void* ws, moe_stream_t stream);
+
+/* FP8 SwiGLU experts read in place from the FP8 rank-major buffer and its
+ * scales (plans with x = FP8, scale_block = 128, inter > 0).  The pages fix
+ * no FP8 GEMM format; this one takes e4m3 weights with one fp32 scale per
+ * 128x128 tile, the 128-column granularity of the dispatched rows.  For every
+ * expert e and row s in [expert_off[e], expert_off[e] + counts[e]), with
+ * X[s, d] = recv[s, d] * recv_scale[s, d/128] and W = code * tile scale:
+ *   h[s, c]  = bf16( silu(X[s] . Wg[e][c]) * (X[s] . Wu[e][c]) )
+ *   hs[s, b] = amax(h[s, 128b .. 128b+127]) / 448 (fp32 quotient; 1 if zero)
+ *   hq[s, c] = e4m3(h[s, c] / hs[s, c/128]), nearest even, saturating at 448
+ *   y[s, c]  = bf16( sum_d hq[s, d] hs[s, d/128] * Wd[e][c, d] )
+ * fp32 accumulation: the tensor cores sum each 128-column block of codes and
+ * the block's scales are applied in fp32.  recv: device e4m3 [T, D];
+ * recv_scale: device fp32 [T, D/128]; w_gate_up: device e4m3 [E, 2I, D] (rows
+ * [0, I) Wg, [I, 2I) Wu) with w_gate_up_scale fp32 [E, 2I/128, D/128];
+ * w_down: device e4m3 [E, D, I] with w_down_scale fp32 [E, D/128, I/128];
+ * h: device bf16 [T, I]; hq: device e4m3 [T, I]; h_scale: device fp32
+ * [T, I/128]; y: device bf16 [T, D].  counts, expert_off and slot_of as
+ * written by moe_route_topk + moe_dispatch (or moe_route_dispatch). */
+MOE_API moe_status moe_expert_swiglu_fp8(const moe_plan* plan, int32_t n, const void* recv,
+                                         const float* recv_scale, const int32_t* counts,
+                                         const int32_t* expert_off, const int32_t* slot_of,
+                                         const void* w_gate_up, const float* w_gate_up_scale,
+                                         const void* w_down, const float* w_down_scale, void* h,
+                                         void* hq, float* h_scale, void* y, void* ws,
+                                         moe_stream_t stream);
 
 /* Combine: out[t, c] = sum_{j=0}^{k-1} topk_w[t, j] * Y[slot_of[t, j], c],
  * accumulated in fp32 with fused multiply-adds in increasing j, then rounded
@@ -210,10 +240,20 @@ MOE_API moe_status moe_layer(const moe_plan* plan, int32_t n, const float* logit
                      const float* x_scale, const void* w_gate_up, const void* w_down,
                      void* out, void* ws, moe_stream_t stream);
 
+/* moe_layer for plans with FP8 experts (x = FP8, inter > 0), which need the
+ * weight scales of moe_expert_swiglu_fp8; moe_layer returns
+ * MOE_ERR_UNSUPPORTED for such plans and this call for any other plan. */
+MOE_API moe_status moe_layer_fp8(const moe_plan* plan, int32_t n, const float* logits,
+                                 const void* x, const float* x_scale, const void* w_gate_up,
+                                 const float* w_gate_up_scale, const void* w_down,
+                                 const float* w_down_scale, void* out, void* ws,
+                                 moe_stream_t stream);
+
 /* Where moe_layer keeps an intermediate inside its workspace, so a caller
  * can read it after the call: returns ws + byte offset, or NULL for an
  * unknown name.  Names: "topk_idx", "topk_w", "counts", "expert_off",
- * "slot_of", "src_of", "recv", "recv_scale", "y", "h". */
+ * "slot_of", "src_of", "recv", "recv_scale", "y", "h", and with FP8 experts
+ * "hq", "h_scale". */
 MOE_API void* moe_layer_buffer(const moe_plan* plan, void* ws, const char* name);
 
 /* Read and clear the device status word of `ws`: synchronises `stream`,

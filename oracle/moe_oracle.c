@@ -285,6 +285,18 @@ int oracle_swiglu_rows(int64_t n_rows, const int32_t* rows, const int32_t* row_e
 
 /* ---------------------------------------------------------------- FP8 experts */
 
+/* e4m3_to_double of every code, filled on first use (the GEMM loops below
+ * decode billions of codes at full layer sizes). */
+static const double* e4m3_values(void) {
+    static double tab[256];
+    static int ready = 0;
+    if (!ready) {
+        for (int c = 0; c < 256; ++c) tab[c] = e4m3_to_double((uint8_t)c);
+        ready = 1;
+    }
+    return tab;
+}
+
 /* Nearest finite e4m3 value to v, ties to the code whose last mantissa bit is
  * 0, magnitudes of 448 and above giving +-448 (saturation instead of NaN;
  * stated as a rule because distances to huge values round to ties).  Below
@@ -353,6 +365,7 @@ int oracle_fp8_gate_up_rows(int64_t n_rows, const int32_t* rows, const int32_t* 
     if (block <= 0 || hidden % block || inter % block) return ORACLE_BAD_ARG;
     int32_t kb = hidden / block;               /* scale blocks along the reduction */
     int32_t rb = 2 * inter / block;            /* scale blocks along an expert's rows */
+    const double* dec = e4m3_values();
     for (int64_t i = 0; i < n_rows; ++i) {
         int64_t s = rows[i];
         int64_t e = row_expert[i];
@@ -364,10 +377,10 @@ int oracle_fp8_gate_up_rows(int64_t n_rows, const int32_t* rows, const int32_t* 
             int64_t cu = (int64_t)inter + c;
             double g = 0.0, u = 0.0;
             for (int32_t d = 0; d < hidden; ++d) {
-                double xv = e4m3_to_double(xr[d]) * (double)xsr[d / block];
-                g += xv * (e4m3_to_double(w[(int64_t)c * hidden + d]) *
+                double xv = dec[xr[d]] * (double)xsr[d / block];
+                g += xv * (dec[w[(int64_t)c * hidden + d]] *
                            (double)wsc[(int64_t)(c / block) * kb + d / block]);
-                u += xv * (e4m3_to_double(w[cu * hidden + d]) *
+                u += xv * (dec[w[cu * hidden + d]] *
                            (double)wsc[(cu / block) * kb + d / block]);
             }
             if (g_out) g_out[s * inter + c] = g;
@@ -389,6 +402,7 @@ int oracle_fp8_down_rows(int64_t n_rows, const int32_t* rows, const int32_t* row
     if (block <= 0 || hidden % block || inter % block) return ORACLE_BAD_ARG;
     int32_t kb = inter / block;
     int32_t rb = hidden / block;
+    const double* dec = e4m3_values();
     for (int64_t i = 0; i < n_rows; ++i) {
         int64_t s = rows[i];
         int64_t e = row_expert[i];
@@ -399,8 +413,8 @@ int oracle_fp8_down_rows(int64_t n_rows, const int32_t* rows, const int32_t* row
         for (int32_t c = 0; c < hidden; ++c) {
             double acc = 0.0;
             for (int32_t d = 0; d < inter; ++d)
-                acc += (e4m3_to_double(hr[d]) * (double)hsr[d / block]) *
-                       (e4m3_to_double(w[(int64_t)c * inter + d]) *
+                acc += (dec[hr[d]] * (double)hsr[d / block]) *
+                       (dec[w[(int64_t)c * inter + d]] *
                         (double)wsc[(int64_t)(c / block) * kb + d / block]);
             y[s * hidden + c] = bf16_from_double(acc);
         }

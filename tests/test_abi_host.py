@@ -75,6 +75,10 @@ def _plan_code(mr, **kw):
     ({"inter": 128}, -2),                     # SwiGLU needs bf16 rows
     ({"inter": 128, "x_dtype": 1, "y_dtype": 1, "out_dtype": 1}, 0),
     ({"inter": 100, "x_dtype": 1, "y_dtype": 1, "out_dtype": 1}, -2),
+    # FP8 experts: FP8 rows with 128-column scales and bf16 Y
+    ({"inter": 128, "x_dtype": 2, "scale_block": 128, "y_dtype": 1, "out_dtype": 1}, 0),
+    ({"inter": 128, "x_dtype": 2, "scale_block": 64, "y_dtype": 1, "out_dtype": 1}, -2),
+    ({"inter": 128, "x_dtype": 2, "scale_block": 128, "y_dtype": 0, "out_dtype": 1}, -2),
     ({"n_max": 1 << 27, "n_experts": 256, "top_k": 8, "n_ranks": 8}, -2),  # T >= 2^31
 ])
 def test_plan_validation(mr, kw, code):
@@ -151,6 +155,34 @@ def test_layer_rejects_bad_arguments_before_its_first_stage(mr):
     p = mr.Plan(64, 256, 8, 2, 2, "bf16", "bf16", "bf16", inter=128)
     assert lib.moe_layer(p.handle, 4, fake, fake, None, None, fake, fake, fake, None) == -1
     assert lib.moe_layer(p.handle, 4, fake, fake, None, fake, odd, fake, fake, None) == -1
+    p.close()
+
+
+def test_fp8_expert_entry_points_validate_on_the_host(mr):
+    fake = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    lib = mr._lib
+    sw8 = lib.moe_expert_swiglu_fp8
+    p = mr.Plan(64, 256, 8, 2, 2, "fp8_e4m3", "bf16", "bf16", scale_block=128, inter=128)
+    args = [fake] * 13 + [fake, None]          # recv .. y, ws, stream
+    assert sw8(p.handle, 4, *args) != -2       # the plan is accepted (the launch then fails)
+    bad = list(args); bad[1] = None            # no recv_scale
+    assert sw8(p.handle, 4, *bad) == -1
+    bad = list(args); bad[10] = odd            # hq misaligned
+    assert sw8(p.handle, 4, *bad) == -1
+    assert sw8(p.handle, 65, *args) == -1      # n > n_max
+    assert sw8(p.handle, 0, *args) == 0        # n = 0 is a no-op
+    # the bf16 expert call and moe_layer refuse FP8 experts; moe_layer_fp8 needs the scales
+    assert lib.moe_expert_swiglu(p.handle, 4, *([fake] * 8), None) == -2
+    assert lib.moe_layer(p.handle, 4, fake, fake, fake, fake, fake, fake, fake, None) == -2
+    assert lib.moe_layer_fp8(p.handle, 4, fake, fake, fake, fake, None, fake, fake, fake, fake,
+                             None) == -1
+    assert lib.moe_layer_buffer(p.handle, fake, b"hq") is not None
+    assert lib.moe_layer_buffer(p.handle, fake, b"h_scale") is not None
+    p.close()
+    p = mr.Plan(64, 256, 8, 2, 2, "bf16", "bf16", "bf16", inter=128)
+    assert sw8(p.handle, 4, *args) == -2       # bf16 experts
+    assert lib.moe_layer_fp8(p.handle, 4, *([fake] * 9), None) == -2
     p.close()
 
 

@@ -51,8 +51,8 @@ MUTANTS = {
     "quant_divisor": ("(float)(amax / 448.0)", "(float)(amax / 240.0)"),
     "quant_signed_amax": ("double a = fabs(bf16_to_double(hb[c]));",
                           "double a = bf16_to_double(hb[c]);"),
-    "fp8_x_scale_dropped": ("double xv = e4m3_to_double(xr[d]) * (double)xsr[d / block];",
-                            "double xv = e4m3_to_double(xr[d]);"),
+    "fp8_x_scale_dropped": ("double xv = dec[xr[d]] * (double)xsr[d / block];",
+                            "double xv = dec[xr[d]];"),
     "fp8_gate_scale_transposed": ("(double)wsc[(int64_t)(c / block) * kb + d / block]);\n"
                                   "                u +=",
                                   "(double)wsc[(int64_t)(d / block) * kb + c / block]);\n"
