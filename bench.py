@@ -137,6 +137,17 @@ def gemm_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
+def fp8_gemm_source_hash() -> str:
+    """Hash of the device code of the FP8 grouped GEMM and H quantisation
+    kernels: fp8_gemm.cu up to its host side, and the device-helper part of
+    the internal header."""
+    h = hashlib.sha256()
+    h.update(_device_part("fp8_gemm.cu",
+                          end=b"// ---------------------------------------------------------------- host side"))
+    h.update(_device_part("moe_internal.cuh", start=_HELPERS))
+    return h.hexdigest()[:16]
+
+
 def recorded_traffic(workload: str, source_hash=kernel_source_hash):
     """DRAM bytes per launch of the dominant kernel from the committed ncu
     summary, if it was taken on the current kernel source (else None)."""
@@ -592,9 +603,11 @@ def run_layer(args, cfg):
     """The MoE layer with SwiGLU experts: route -> dispatch -> grouped GEMMs
     (tcgen05) -> combine.  The roofline line is the grouped GEMM against
     whichever peak bounds it: the weight stream (HBM) at small batches, the
-    tensor cores once enough rows share each expert's weights.  Expert weights (5.6 GB at the layer shape) are drawn on
+    tensor cores once enough rows share each expert's weights.  Expert
+    weights (5.6 GB in bf16, 2.8 GB in FP8 at the layer shape) are drawn on
     the device from a seeded generator with the workload's N(0, w_std)
-    distribution; parity tests draw them on the host."""
+    distribution, and for FP8 experts quantised per 128x128 tile there;
+    parity tests draw them on the host."""
     world, rank, local = init_dist()
     import combine_moe_route_11_b200 as mr
     torch.cuda.set_device(local)
@@ -602,26 +615,42 @@ def run_layer(args, cfg):
     stream = torch.cuda.current_stream(dev)
     n, E, D, I, k = cfg.n, cfg.n_experts, cfg.hidden, cfg.inter, cfg.top_k
     plan = mr.Plan.from_config(cfg, n_max=n)
+    fp8 = plan.fp8_experts
     inp = workloads.make_inputs(cfg, seed=rank, n=n, with_weights=False)
     logits, x = inp["logits"].to(dev), inp["x"].to(dev)
+    xs = inp["x_scale"].to(dev) if inp["x_scale"] is not None else None
     gen = torch.Generator(device=dev).manual_seed(1000 + rank)
-    wgu = torch.empty(E, 2 * I, D, dtype=torch.bfloat16, device=dev)
-    wd = torch.empty(E, D, I, dtype=torch.bfloat16, device=dev)
+    wdt = torch.uint8 if fp8 else torch.bfloat16
+    wgu = torch.empty(E, 2 * I, D, dtype=wdt, device=dev)
+    wd = torch.empty(E, D, I, dtype=wdt, device=dev)
+    sgu = torch.empty(E, 2 * I // 128, D // 128, device=dev) if fp8 else None
+    sd = torch.empty(E, D // 128, I // 128, device=dev) if fp8 else None
     for e in range(E):
-        wgu[e] = (torch.randn(2 * I, D, generator=gen, device=dev) * cfg.w_std).to(torch.bfloat16)
-        wd[e] = (torch.randn(D, I, generator=gen, device=dev) * cfg.w_std).to(torch.bfloat16)
+        a = torch.randn(2 * I, D, generator=gen, device=dev) * cfg.w_std
+        c = torch.randn(D, I, generator=gen, device=dev) * cfg.w_std
+        if fp8:
+            wgu[e], sgu[e] = workloads.quantise_fp8_tiles(a, 128)
+            wd[e], sd[e] = workloads.quantise_fp8_tiles(c, 128)
+        else:
+            wgu[e], wd[e] = a.to(torch.bfloat16), c.to(torch.bfloat16)
+    del a, c
     ws = plan.new_workspace(dev)
     b = plan.new_buffers(n, dev)
 
     def route_dispatch():
         # the call moe_layer makes: one launch at n <= 1024, else two
-        mr.moe_route_dispatch(plan, logits, x, None, b["topk_idx"], b["topk_w"], b["counts"],
-                              b["expert_off"], b["recv"], None, b["slot_of"], b["src_of"], ws,
-                              stream)
+        mr.moe_route_dispatch(plan, logits, x, xs, b["topk_idx"], b["topk_w"], b["counts"],
+                              b["expert_off"], b["recv"], b.get("recv_scale"), b["slot_of"],
+                              b["src_of"], ws, stream)
 
     def expert():
-        mr.moe_expert_swiglu(plan, n, b["recv"], b["counts"], b["expert_off"], wgu, wd, b["h"],
-                             b["y"], ws, stream)
+        if fp8:
+            mr.moe_expert_swiglu_fp8(plan, n, b["recv"], b["recv_scale"], b["counts"],
+                                     b["expert_off"], b["slot_of"], wgu, sgu, wd, sd, b["h"],
+                                     b["hq"], b["h_scale"], b["y"], ws, stream)
+        else:
+            mr.moe_expert_swiglu(plan, n, b["recv"], b["counts"], b["expert_off"], wgu, wd,
+                                 b["h"], b["y"], ws, stream)
 
     def combine():
         mr.moe_combine(plan, b["y"], b["topk_w"], b["slot_of"], b["out"], ws, stream)
@@ -663,9 +692,20 @@ def run_layer(args, cfg):
     ms_step = reduce_max(r0.elapsed_time(r1), dev) / args.steps
     rows = n * k
     flops = 2.0 * rows * (2 * I * D + D * I)
-    wbytes = (wgu.numel() + wd.numel()) * 2
-    # activations the two GEMMs must move: X rows read, H written and read, Y written
-    abytes = rows * (D * 2 + 2 * I * 2 + D * 2)
+    if fp8:
+        # e4m3 weights plus one fp32 scale per 128x128 tile
+        wbytes = wgu.numel() + wd.numel() + (sgu.numel() + sd.numel()) * 4
+        # activations the layer must move: X codes + scales read, Hq codes +
+        # scales written and read, Y written (the bf16 H that GEMM1 hands to
+        # the quantisation kernel is this implementation's extra round trip
+        # and is not counted)
+        abytes = rows * (D + D // 32 + 2 * (I + I // 32) + D * 2)
+        kernel = "expert_gemm (GEMM1 + H quantisation + GEMM2)"
+    else:
+        wbytes = (wgu.numel() + wd.numel()) * 2
+        # activations the two GEMMs must move: X rows read, H written and read, Y written
+        abytes = rows * (D * 2 + 2 * I * 2 + D * 2)
+        kernel = "expert_gemm (GEMM1 + GEMM2)"
     t_gemm = kern_ms["expert_gemm"] * 1e-3
     tfs = flops / t_gemm / 1e12
     gbs = (wbytes + abytes) / t_gemm / 1e9
@@ -676,20 +716,24 @@ def run_layer(args, cfg):
     except OSError:
         pass
     peak = float(peaks.get("bf16_tflops_sustained", 1400.0))
+    peak_kind = "measured sustained" if peaks else "fallback"
+    if fp8:
+        # no measured e4m3 peak: the bf16 one times the nominal e4m3 / bf16 ratio (4.5 / 2.25)
+        peak *= 2.0
+        peak_kind += " bf16 x 2 (nominal e4m3/bf16 ratio)"
     hbm_peak, _ = read_peaks()
     # the roofline is whichever resource needs longer at its measured peak
-    tensor_line = {"bound": "tensor", "kernel": "expert_gemm (GEMM1 + GEMM2)",
-                   "achieved": tfs, "peak": peak,
-                   "peak_kind": "measured sustained" if peaks else "fallback",
+    tensor_line = {"bound": "tensor", "kernel": kernel,
+                   "achieved": tfs, "peak": peak, "peak_kind": peak_kind,
                    "unit": "TFLOP/s", "frac": tfs / peak, "traffic": None}
-    full_shape = (n, E, D, I) == (workloads.CONFIGS["layer"].n, workloads.CONFIGS["layer"].n_experts,
-                                  workloads.CONFIGS["layer"].hidden,
-                                  workloads.CONFIGS["layer"].inter)
-    hbm_line = {"bound": "hbm", "kernel": "expert_gemm (GEMM1 + GEMM2)",
+    base = workloads.CONFIGS[cfg.name]
+    full_shape = (n, E, D, I) == (base.n, base.n_experts, base.hidden, base.inter)
+    record = ("layer_fp8", fp8_gemm_source_hash) if fp8 else ("layer", gemm_source_hash)
+    hbm_line = {"bound": "hbm", "kernel": kernel,
                 "achieved": gbs, "peak": hbm_peak,
                 "peak_kind": "measured" if peaks else "fallback",
                 "unit": "GB/s", "frac": gbs / hbm_peak,
-                "traffic": recorded_traffic("layer", gemm_source_hash) if full_shape else None,
+                "traffic": recorded_traffic(*record) if full_shape else None,
                 "algorithmic_bytes": wbytes + abytes}
     hbm_bound = (wbytes + abytes) / (hbm_peak * 1e9) >= flops / (peak * 1e12)
     roofline, other = (hbm_line, tensor_line) if hbm_bound else (tensor_line, hbm_line)
@@ -698,16 +742,20 @@ def run_layer(args, cfg):
             "metric": "MoE layer tokens/s (route + dispatch + SwiGLU grouped GEMM + combine)",
             "value": world * n / (ms_step * 1e-3), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "fp8_e4m3 (fp32 accumulate)" if fp8 else "bf16",
             "data": "synthetic (expert weights drawn on the device, seeded)",
-            "config": {"workload": describe(cfg, n) + f", SwiGLU I={I}, W~N(0,{cfg.w_std})",
-                       "l2": "each step streams 5.6 GB of weights (> 40x L2)"},
+            "config": {"workload": describe(cfg, n) + f", SwiGLU I={I}, W~N(0,{cfg.w_std})"
+                       + (" as e4m3 with an fp32 scale per 128x128 tile" if fp8 else ""),
+                       "l2": f"each step streams {wbytes / 1e9:.1f} GB of weights (> 20x L2)"},
             "kernel_us": {kk: v * 1e3 for kk, v in kern_ms.items()},
             "roofline": roofline,
             "roofline_other": other,
             "weight_stream_gbs": wbytes / (kern_ms["expert_gemm"] * 1e-3) / 1e9,
             "weight_stream_frac_of_hbm": wbytes / (kern_ms["expert_gemm"] * 1e-3) / 1e9 / hbm_peak,
-            "gpu_launches": (4 if n <= mr.FUSED_MAX_TOKENS else 5) * args.steps,
+            # route(+dispatch), GEMM1, [H quantisation,] GEMM2, combine
+            "gpu_launches": ((4 if n <= mr.FUSED_MAX_TOKENS else 5) + (1 if fp8 else 0))
+            * args.steps,
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)

@@ -23,7 +23,8 @@ from __future__ import annotations
 import dataclasses
 import torch
 
-__all__ = ["Config", "CONFIGS", "make_inputs", "as_numpy_bits", "DTYPE_BYTES"]
+__all__ = ["Config", "CONFIGS", "make_inputs", "as_numpy_bits", "DTYPE_BYTES",
+           "quantise_fp8_tiles"]
 
 # Element size in bytes of each activation encoding the library accepts.
 DTYPE_BYTES = {"f32": 4, "bf16": 2, "fp8_e4m3": 1}
@@ -92,7 +93,7 @@ def _quantise_fp8_blocks(xf: torch.Tensor, block: int):
     return q.contiguous(), scale.to(torch.float32).contiguous()
 
 
-def _quantise_fp8_tiles(wf: torch.Tensor, block: int):
+def quantise_fp8_tiles(wf: torch.Tensor, block: int):
     """Per-(block x block tile) amax scaling of a weight matrix to e4m3 codes."""
     r, c = wf.shape
     wb = wf.view(r // block, block, c // block, block)
@@ -145,9 +146,9 @@ def make_inputs(cfg: Config, seed: int = 0, n: int | None = None,
         sgu = torch.empty(e, 2 * i // b, d // b, dtype=torch.float32)
         sd = torch.empty(e, d // b, i // b, dtype=torch.float32)
         for ex in range(e):
-            wgu[ex], sgu[ex] = _quantise_fp8_tiles(torch.randn(2 * i, d, generator=g) * cfg.w_std, b)
+            wgu[ex], sgu[ex] = quantise_fp8_tiles(torch.randn(2 * i, d, generator=g) * cfg.w_std, b)
         for ex in range(e):
-            wd[ex], sd[ex] = _quantise_fp8_tiles(torch.randn(d, i, generator=g) * cfg.w_std, b)
+            wd[ex], sd[ex] = quantise_fp8_tiles(torch.randn(d, i, generator=g) * cfg.w_std, b)
         out.update(w_gate_up=wgu, w_down=wd, w_gate_up_scale=sgu, w_down_scale=sd)
     elif with_weights:
         e, d, i = cfg.n_experts, cfg.hidden, cfg.inter
