@@ -399,6 +399,32 @@ def pin_fp8_gate_up_equals_bf16_with_unit_scales(o):
     assert np.array_equal(h8, h16)
 
 
+def pin_run_path_fp8_layer(o):
+    """The composed FP8 expert path keeps its invariants: H codes times their
+    scale reproduce H to within half an e4m3 step of the block, every block
+    scale is its amax / 448, Y equals the down projection of the quantised H,
+    and rows outside the filled slots stay zero."""
+    import workloads
+    cfg = workloads.CONFIGS["layer_fp8"].replace(n=24, hidden=256, inter=256, n_experts=4,
+                                                 top_k=2, n_ranks=2)
+    inp = {kk: workloads.as_numpy_bits(v) for kk, v in workloads.make_inputs(cfg).items()}
+    res = o.run_path(cfg, inp)
+    fs = np.sort(res["slot_of"].reshape(-1))
+    hv = _bf16_val(res["h"][fs])
+    dq = _e4m3_val(res["hq"][fs]) * np.repeat(res["h_scale"][fs].astype(np.float64), 128, axis=1)
+    amax = np.abs(hv).reshape(len(fs), -1, 128).max(axis=2)
+    sc = res["h_scale"][fs].astype(np.float64)
+    assert np.allclose(sc, np.where(amax > 0, amax / 448.0, 1.0), rtol=2 ** -23, atol=0)
+    # an e4m3 step is at most 2^-3 of the value (normal) or 2^-9 of the block scale (subnormal)
+    step = np.maximum(np.abs(hv) * 2.0 ** -3, np.repeat(sc, 128, axis=1) * 2.0 ** -9)
+    assert np.all(np.abs(dq - hv) <= 0.5 * step + 1e-300)
+    expert = res["topk_idx"].reshape(-1)[res["src_of"][fs]]
+    y = o.fp8_down_rows(fs, expert, res["hq"], res["h_scale"], inp["w_down"], inp["w_down_scale"])
+    assert np.array_equal(y[fs], res["y"][fs])
+    unfilled = np.setdiff1d(np.arange(res["y"].shape[0]), fs)
+    assert np.all(res["y"][unfilled] == 0) and np.all(res["hq"][unfilled] == 0)
+
+
 # ------------------------------------------------------------------ combine
 def pin_combine_identity_roundtrip(o):
     """combine(dispatch(x)) with identity experts and renormalised weights is

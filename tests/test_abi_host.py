@@ -267,3 +267,51 @@ def test_binding_checks_slot_indexed_buffers(mr):
         mr.moe_layer(p, torch.zeros(n, 8), bf(n), None, None, wd, out,
                      torch.zeros(p.layer_workspace_bytes, dtype=torch.uint8))
     p.close()
+
+
+def test_binding_checks_fp8_expert_buffers(mr):
+    """moe_expert_swiglu_fp8 / moe_layer_fp8 reject mistyped or short weights,
+    scales and intermediates before any pointer reaches the library."""
+    import torch
+    n, E, D, I = 16, 8, 256, 128
+    p = mr.Plan(64, D, E, 2, 2, "fp8_e4m3", "bf16", "bf16", scale_block=128, inter=I)
+    assert p.fp8_experts
+    T = p.recv_rows(n)
+    ws = torch.zeros(p.workspace_bytes, dtype=torch.uint8)
+    u8 = lambda *s: torch.zeros(*s, dtype=torch.uint8)  # noqa: E731
+    f32 = lambda *s: torch.zeros(*s, dtype=torch.float32)  # noqa: E731
+    bf = lambda *s: torch.zeros(*s, dtype=torch.bfloat16)  # noqa: E731
+    i32 = lambda *s: torch.zeros(*s, dtype=torch.int32)  # noqa: E731
+    args = dict(recv=u8(T, D), recv_scale=f32(T, D // 128), counts=i32(E), expert_off=i32(E + 1),
+                slot_of=i32(n, 2), w_gate_up=u8(E, 2 * I, D), w_gate_up_scale=f32(E, 2 * I // 128, D // 128),
+                w_down=u8(E, D, I), w_down_scale=f32(E, D // 128, I // 128), h=bf(T, I), hq=u8(T, I),
+                h_scale=f32(T, I // 128), y=bf(T, D))
+
+    def call(**over):
+        a = dict(args, **over)
+        mr.moe_expert_swiglu_fp8(p, n, a["recv"], a["recv_scale"], a["counts"], a["expert_off"],
+                                 a["slot_of"], a["w_gate_up"], a["w_gate_up_scale"], a["w_down"],
+                                 a["w_down_scale"], a["h"], a["hq"], a["h_scale"], a["y"], ws)
+
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        call()                                               # every check passes
+    with pytest.raises(TypeError, match="w_gate_up: dtype"):
+        call(w_gate_up=bf(E, 2 * I, D))
+    with pytest.raises(ValueError, match="w_down_scale: shape"):
+        call(w_down_scale=f32(E, D // 128, I // 64))
+    with pytest.raises(ValueError, match="hq: shape"):
+        call(hq=u8(T - 1, I))
+    with pytest.raises(ValueError, match="h_scale: shape"):
+        call(h_scale=f32(T, I // 64))
+    with pytest.raises(ValueError, match="recv_scale: shape"):
+        call(recv_scale=f32(T, 1))
+    with pytest.raises(ValueError, match="w_gate_up_scale: required"):
+        call(w_gate_up_scale=None)
+    lws = torch.zeros(p.layer_workspace_bytes, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="w_down: shape"):
+        mr.moe_layer_fp8(p, f32(n, E), u8(n, D), f32(n, D // 128), args["w_gate_up"],
+                         args["w_gate_up_scale"], u8(E, D, I // 2), args["w_down_scale"],
+                         bf(n, D), lws)
+    buf = p.new_buffers(0, device="cpu")
+    assert set(("hq", "h_scale", "h", "y")) <= set(buf)
+    p.close()
