@@ -6,7 +6,8 @@
 
 A step is one pass of the hot path over one batch of synthetic tokens that is
 already resident in HBM: route (top-k + counts + scan) -> dispatch -> combine,
-three kernel launches.  The expert output Y that combine reads is produced
+three kernel launches (two up to 1024 tokens, where route and dispatch run as
+one launch).  The expert output Y that combine reads is produced
 once before timing by the identity expert (FP8 rows dequantised to bf16);
 it is an input of the dispatch+combine metric, like x.  No step finds its
 inputs in L2: a step moves more than 4x the L2 size, or else enough buffer
@@ -14,13 +15,19 @@ sets rotate that 4x L2 of traffic separates two uses of a set.  Steps run
 back to back; the K-step region is timed with CUDA events on the launching
 stream and reduced with MAX across ranks.  Kernel durations (for the
 roofline) come from a separate pass with events between the kernels, which
-would otherwise break the programmatic-launch overlap between them.  With N > 1 every rank runs an independent
-replica on its own GPU (the path has no cross-GPU step on one GPU's virtual
+would otherwise break the programmatic-launch overlap between them.  With
+N > 1 every rank runs an independent replica on its own GPU (the path has no cross-GPU step on one GPU's virtual
 ranks), so scaling is weak and value = all ranks' tokens / max time.
 
 `e2e` times the public call a user makes, moe_layer, with pinned host
 buffers: host->device copies of logits, x and scales, the layer (route,
 dispatch, identity expert, combine) and the device->host copy of out.
+
+`--workload layer` and `--workload layer_fp8` time the MoE layer with SwiGLU
+experts instead (bf16, or FP8 with 128-column row scales and 128x128 weight-tile
+scales): route + dispatch -> grouped GEMMs on the tensor cores -> combine.
+Their roofline line is the grouped GEMMs against HBM or the tensor peak,
+whichever binds at the batch.
 """
 from __future__ import annotations
 
