@@ -302,6 +302,15 @@ def reduce_max(value: float, device) -> float:
     return float(t.item())
 
 
+def reduce_max_list(values, device) -> list:
+    """Element-wise max over ranks of a list of floats."""
+    if not (dist.is_available() and dist.is_initialized()):
+        return list(values)
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
 def job_throughput(world: int, tokens_per_rank: int, max_ms_per_step: float) -> float:
     """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
     return world * tokens_per_rank / (max_ms_per_step * 1e-3)
@@ -316,62 +325,233 @@ def barrier(device):
 
 
 # ------------------------------------------------------------------ CPU oracle timing
-def time_oracle(cfg, budget_s: float, max_tokens: int, seed: int = 0):
-    """Tokens/s of the CPU oracle (route, dispatch, identity expert, combine)
-    on a sample sized to take about budget_s seconds."""
+def host_cpu() -> dict:
+    """The host CPU the oracle runs on: model name and cores."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.lower().startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        avail = len(os.sched_getaffinity(0))
+    except AttributeError:
+        avail = os.cpu_count() or 1
+    return {"cpu_model": model, "cores_available": avail, "nproc": os.cpu_count()}
+
+
+# most oracle worker processes started at once (each holds its slice's buffers)
+MAX_ORACLE_WORKERS = 64
+
+_CFG_FIELDS = ("n_experts", "top_k", "n_ranks", "inter", "x_dtype", "y_dtype", "out_dtype",
+               "scale_block")
+
+
+class OracleCores:
+    """The CPU oracle on several host cores at once: one worker process per
+    core (oracle/timing_worker.py), each running the unchanged
+    single-threaded oracle on its own contiguous slice of the batch's tokens
+    as an independent sub-batch.  Workers load their slice first; a step
+    sends "go" to all of them and lasts until the slowest one answers."""
+
+    def __init__(self, cfg, inp_np: dict, workers: int):
+        import tempfile
+        import numpy as np
+        n = inp_np["logits"].shape[0]
+        self.workers = max(1, min(workers, n))
+        self.tokens = n
+        self.tmp = tempfile.TemporaryDirectory(prefix="moe_oracle_")
+        cfg_path = os.path.join(self.tmp.name, "cfg.json")
+        with open(cfg_path, "w") as f:
+            json.dump({k: getattr(cfg, k) for k in _CFG_FIELDS}, f)
+        bounds = [n * i // self.workers for i in range(self.workers + 1)]
+        self.procs = []
+        for i in range(self.workers):
+            path = os.path.join(self.tmp.name, f"slice{i}.npz")
+            np.savez(path, **{k: inp_np[k][bounds[i]:bounds[i + 1]]
+                              for k in ("logits", "x", "x_scale") if inp_np.get(k) is not None})
+            self.procs.append(subprocess.Popen(
+                [sys.executable, "-m", "oracle.timing_worker", path, cfg_path], cwd=ROOT,
+                stdin=subprocess.PIPE, stdout=subprocess.PIPE, text=True))
+        for p in self.procs:
+            if p.stdout.readline().strip() != "ready":
+                self.close()
+                raise RuntimeError("an oracle worker failed to start")
+
+    def step(self) -> float:
+        """Wall seconds of one pass of every worker over its slice."""
+        t0 = time.perf_counter()
+        for p in self.procs:
+            p.stdin.write("go\n")
+            p.stdin.flush()
+        for p in self.procs:
+            float(p.stdout.readline())
+        return time.perf_counter() - t0
+
+    def close(self):
+        for p in self.procs:
+            try:
+                p.stdin.write("quit\n")
+                p.stdin.flush()
+                p.wait(timeout=30)
+            except (OSError, subprocess.TimeoutExpired, ValueError):
+                p.kill()
+        self.tmp.cleanup()
+
+
+def oracle_inputs(cfg, n: int, seed: int = 0) -> dict:
+    return {k: workloads.as_numpy_bits(v) for k, v in
+            workloads.make_inputs(cfg, seed=seed, n=n).items()}
+
+
+def oracle_seconds_per_token(cfg, n_cal: int = 16) -> float:
+    """Single-core seconds per token of the oracle's whole path (calibration)."""
     import oracle
-    cal_n = min(64, max_tokens)
-    inp = {k: workloads.as_numpy_bits(v) for k, v in
-           workloads.make_inputs(cfg, seed=seed, n=cal_n).items()}
+    inp = oracle_inputs(cfg, n_cal)
     t0 = time.perf_counter()
     oracle.run_path(cfg, inp)
-    per_tok = (time.perf_counter() - t0) / cal_n
+    return (time.perf_counter() - t0) / n_cal
+
+
+def time_oracle(cfg, budget_s: float, max_tokens: int, seed: int = 0):
+    """Tokens/s of the CPU oracle (route, dispatch, identity expert, combine)
+    on one core, on a sample sized to take about budget_s seconds."""
+    import oracle
+    per_tok = oracle_seconds_per_token(cfg)
     n = int(max(1, min(max_tokens, budget_s / max(per_tok, 1e-9))))
-    inp = {k: workloads.as_numpy_bits(v) for k, v in
-           workloads.make_inputs(cfg, seed=seed, n=n).items()}
+    inp = oracle_inputs(cfg, n, seed)
     t0 = time.perf_counter()
     oracle.run_path(cfg, inp)
     dt = time.perf_counter() - t0
     return n, dt
 
 
+def cpu_baseline_leg(cfg, n: int) -> dict:
+    """The oracle timed on the host: single-threaded on a ~6 s sample, and on
+    all host cores (up to MAX_ORACLE_WORKERS) over the whole N-token batch."""
+    host = host_cpu()
+    nt1, dt1 = time_oracle(cfg, budget_s=6.0, max_tokens=n)
+    workers = min(host["cores_available"], MAX_ORACLE_WORKERS)
+    pool = OracleCores(cfg, oracle_inputs(cfg, n), workers)
+    try:
+        pool.step()  # first touch of every buffer
+        walls = [pool.step() for _ in range(3)]
+    finally:
+        pool.close()
+    wall = statistics.median(walls)
+    path = ("the oracle's whole path (route, counts, offsets, slots, dispatch, identity "
+            "expert, combine), unchanged single-threaded C")
+    return {"value": n / wall, "unit": "tokens/s", "cores": pool.workers, "kind": "oracle",
+            "sample": (f"all {n} tokens of the batch, split into {pool.workers} contiguous "
+                       f"slices run as independent sub-batches by {pool.workers} worker "
+                       f"processes at once; median of 3 passes ({wall:.2f} s each) after one "
+                       f"untimed pass; {path}"),
+            **host,
+            "single_thread": {"value": nt1 / dt1, "unit": "tokens/s", "cores": 1,
+                              "sample": f"{nt1} of the {n} tokens in one process, one pass "
+                                        f"in {dt1:.1f} s"}}
+
+
 def run_reference(args, cfg):
+    """The oracle as the reference arm, on the host cores: every step runs a
+    bounded sample of the batch's tokens split over the workers, and the
+    line reports the measured time of those steps."""
     world, rank, _ = init_dist()
     if rank != 0:
         return
+    host = host_cpu()
+    workers = min(host["cores_available"], MAX_ORACLE_WORKERS)
     n_steps = args.steps + args.warmup
-    per_step_budget = max(0.02, 90.0 / max(1, n_steps))
-    import oracle
-    cal = {k: workloads.as_numpy_bits(v) for k, v in
-           workloads.make_inputs(cfg, seed=0, n=16).items()}
-    t0 = time.perf_counter()
-    oracle.run_path(cfg, cal)
-    per_tok = (time.perf_counter() - t0) / 16
-    n = int(max(1, min(cfg.n, per_step_budget / max(per_tok, 1e-9))))
-    inp = {k: workloads.as_numpy_bits(v) for k, v in
-           workloads.make_inputs(cfg, seed=0, n=n).items()}
-    for _ in range(args.warmup):
-        oracle.run_path(cfg, inp)
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        oracle.run_path(cfg, inp)
-    dt = time.perf_counter() - t0
+    per_step_budget = max(0.05, 90.0 / max(1, n_steps))
+    per_tok = oracle_seconds_per_token(cfg)
+    n = int(max(1, min(cfg.n, per_step_budget * workers / max(per_tok, 1e-9))))
+    pool = OracleCores(cfg, oracle_inputs(cfg, n), workers)
+    try:
+        for _ in range(args.warmup):
+            pool.step()
+        walls = [pool.step() for _ in range(args.steps)]
+    finally:
+        pool.close()
+    dt = sum(walls)
     value = n * args.steps / dt
-    sample = (f"{n} of the {cfg.n} tokens per step, the oracle's whole path "
-              f"(route, counts, offsets, slots, dispatch, identity expert, combine)")
+    sample = (f"{n} of the {cfg.n} tokens per step (the first {n} of the seed-0 batch), split "
+              f"into {pool.workers} contiguous slices run as independent sub-batches by "
+              f"{pool.workers} worker processes at once; the oracle's whole path (route, counts, "
+              f"offsets, slots, dispatch, identity expert, combine), unchanged single-threaded C")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": dt / args.steps * 1e3 * cfg.n / n, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "ms_per_step": dt / args.steps * 1e3, "tokens_per_step": n,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64 (oracle arithmetic)", "data": "synthetic",
             "config": step_config(cfg, cfg.n, buffer_sets(cfg, cfg.n), args.gpus),
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                             "sample": sample},
+            "step_ms": percentiles([w * 1e3 for w in walls]),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": pool.workers,
+                             "kind": "oracle", "sample": sample, **host},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
+def percentiles(xs) -> dict:
+    """p10 / median / p90 of a list (nearest-rank on the sorted values)."""
+    v = sorted(xs)
+    if not v:
+        return {}
+    pick = lambda q: v[min(len(v) - 1, max(0, int(round(q * (len(v) - 1)))))]  # noqa: E731
+    return {"n": len(v), "p10": pick(0.1), "p50": statistics.median(v), "p90": pick(0.9),
+            "min": v[0], "max": v[-1]}
+
+
 # ------------------------------------------------------------------ GPU arm
+# The K-step region repeats back to back until this much work was timed, so
+# that the clock sampler sees the GPU under load and regions can be compared.
+MIN_WINDOW_S = 0.1
+MAX_REPEATS = 2000
+
+
+def timed_regions(region, stream, dev, steps: int):
+    """Time region() -- K steps -- R times back to back, one CUDA event pair
+    per region on the launching stream, bracketed by a barrier and a device
+    synchronisation on both sides.  R is chosen from one untimed region so
+    that the R regions last at least MIN_WINDOW_S.  Returns the regions'
+    milliseconds (each the max over ranks) and the wall-clock window."""
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    region()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    one_ms = reduce_max(e0.elapsed_time(e1), dev)
+    repeats = int(min(MAX_REPEATS, max(1, -(-MIN_WINDOW_S * 1e3 // max(one_ms, 1e-3)))))
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(repeats + 1)]
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    t_start = time.time()
+    ev[0].record(stream)
+    for r in range(repeats):
+        region()
+        ev[r + 1].record(stream)
+    torch.cuda.synchronize(dev)
+    t_end = time.time()
+    barrier(dev)
+    times = reduce_max_list([ev[r].elapsed_time(ev[r + 1]) for r in range(repeats)], dev)
+    return times, t_start, t_end
+
+
+def path_dtype(cfg) -> str:
+    """What the path computes in: the row encoding it moves, the expert-output
+    and output types, and the accumulation type of the combine."""
+    rows = {"f32": "fp32", "bf16": "bf16", "fp8_e4m3": "fp8_e4m3"}[cfg.x_dtype]
+    if cfg.scale_block:
+        rows += f" + fp32 scale per {cfg.scale_block} cols"
+    names = {"f32": "fp32", "bf16": "bf16"}
+    return (f"{rows} rows moved as bytes, {names[cfg.y_dtype]} Y / {names[cfg.out_dtype]} out, "
+            f"fp32 accumulate")
+
+
 def time_e2e(mr, plan, inp, n, out_dtype, dev, stream, steps, world):
     """Steps through the public moe_layer call, each with the host->device
     copy of its inputs from pinned memory and the device->host copy of its
@@ -526,7 +706,9 @@ def run_ours(args, cfg):
     torch.cuda.synchronize(dev)
     kern_ms = {name: sum(e[j].elapsed_time(e[j + 1]) for e in ev) / k_steps
                for j, (name, _) in enumerate(stages)}
-    # pass 2: K steps back to back, events only around the region
+    # pass 2: the K-step region back to back, events only around each region;
+    # the region repeats until >= MIN_WINDOW_S of timed work, so that the
+    # clock samples fall inside it and the spread between regions shows
     sampler = ClockSampler(local)
     sampler.wait_first()
     for i in range(args.warmup):
@@ -542,26 +724,35 @@ def run_ours(args, cfg):
             graphs.append(g)
         for i in range(args.warmup):
             graphs[i % n_sets].replay()
-    r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(dev)
+
+    def region():
+        for i in range(args.steps):
+            if graphs:
+                graphs[i % n_sets].replay()
+            else:
+                step(sets[i % n_sets])
+
+    region_ms, t_start, t_end = timed_regions(region, stream, dev, args.steps)
+    clocks = sampler.stop(t_start, t_end)
+    # per-step distribution: >= 100 steps with an event after every step (the
+    # events cut the launch overlap across step boundaries, so these read a
+    # little above the back-to-back steps)
+    n_dist = max(100, min(args.steps, 1000))
+    dev_ev = [torch.cuda.Event(enable_timing=True) for _ in range(n_dist + 1)]
     torch.cuda.synchronize(dev)
-    t_start = time.time()
-    r0.record(stream)
-    for i in range(args.steps):
+    dev_ev[0].record(stream)
+    for i in range(n_dist):
         if graphs:
             graphs[i % n_sets].replay()
         else:
             step(sets[i % n_sets])
-    r1.record(stream)
+        dev_ev[i + 1].record(stream)
     torch.cuda.synchronize(dev)
-    t_end = time.time()
-    barrier(dev)
-    clocks = sampler.stop(t_start, t_end)
+    per_step = [dev_ev[i].elapsed_time(dev_ev[i + 1]) for i in range(n_dist)]
     for st in sets:
         if mr.moe_get_status(plan, st["ws"], stream) != 0:
             raise RuntimeError("device status set during timing")
-    total_ms = reduce_max(r0.elapsed_time(r1), dev)
-    ms_step = total_ms / args.steps
+    ms_step = statistics.median(region_ms) / args.steps
     peak, peak_kind = read_peaks()
     dom = max((k for k in kern_ms if k != "route"), key=lambda k: kern_ms[k])
     achieved = nb[dom] / (kern_ms[dom] * 1e-3) / 1e9
@@ -577,19 +768,18 @@ def run_ours(args, cfg):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        nt, dt = time_oracle(cfg, budget_s=12.0, max_tokens=n)
-        cpu = {"value": nt / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-               "sample": f"{nt} of the {n} tokens of this workload, one pass of the oracle's "
-                         f"whole path (route, counts, offsets, slots, dispatch, identity expert, "
-                         f"combine) in {dt:.1f} s, single-threaded C"}
+        cpu = cpu_baseline_leg(cfg, n)
 
     if rank == 0:
         line = {
             "metric": METRIC, "value": job_throughput(world, n, ms_step), "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f32", "data": "synthetic",
+            "dtype": path_dtype(cfg), "data": "synthetic",
             "config": step_config(cfg, n, n_sets, world, args.graph),
+            "repeats": len(region_ms),
+            "region_ms_per_step": percentiles([r / args.steps for r in region_ms]),
+            "step_ms": dict(percentiles(per_step), how="one event after every step"),
             "hbm_gbs": step_gbs, "hbm_pct_of_peak": 100.0 * step_gbs / peak,
             "kernel_us": {k: v * 1e3 for k, v in kern_ms.items()},
             "algorithmic_bytes": nb,
@@ -681,22 +871,17 @@ def run_layer(args, cfg):
                for j, nm in enumerate(names)}
     sampler = ClockSampler(local)
     sampler.wait_first()
-    r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(dev)
-    torch.cuda.synchronize(dev)
-    t_start = time.time()
-    r0.record(stream)
-    for _ in range(args.steps):
-        for f in stages:
-            f()
-    r1.record(stream)
-    torch.cuda.synchronize(dev)
-    t_end = time.time()
-    barrier(dev)
+
+    def region():
+        for _ in range(args.steps):
+            for f in stages:
+                f()
+
+    region_ms, t_start, t_end = timed_regions(region, stream, dev, args.steps)
     clocks = sampler.stop(t_start, t_end)
     if mr.moe_get_status(plan, ws, stream) != 0:
         raise RuntimeError("device status set during timing")
-    ms_step = reduce_max(r0.elapsed_time(r1), dev) / args.steps
+    ms_step = statistics.median(region_ms) / args.steps
     rows = n * k
     flops = 2.0 * rows * (2 * I * D + D * I)
     if fp8:
@@ -750,8 +935,11 @@ def run_layer(args, cfg):
             "value": world * n / (ms_step * 1e-3), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "fp8_e4m3 (fp32 accumulate)" if fp8 else "bf16",
+            "dtype": ("fp8_e4m3 rows and weights with fp32 block scales, bf16 H/Y/out, fp32 "
+                      "accumulate" if fp8 else "bf16 rows, weights, H, Y and out, fp32 accumulate"),
             "data": "synthetic (expert weights drawn on the device, seeded)",
+            "repeats": len(region_ms),
+            "region_ms_per_step": percentiles([r / args.steps for r in region_ms]),
             "config": {"workload": describe(cfg, n) + f", SwiGLU I={I}, W~N(0,{cfg.w_std})"
                        + (" as e4m3 with an fp32 scale per 128x128 tile" if fp8 else ""),
                        "l2": f"each step streams {wbytes / 1e9:.1f} GB of weights (> 20x L2)"},

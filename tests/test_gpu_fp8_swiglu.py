@@ -200,6 +200,36 @@ def test_fp8_swiglu_tile_shapes_from_designed_counts():
     assert list(b["counts"].numpy()) == counts
 
 
+def test_fp8_swiglu_layer_config():
+    """The FP8 layer workload exactly as configured and benchmarked: N = 1024,
+    D = 7168, E = 64, k = 8, R = 8, I = 2048, route and dispatch in one
+    launch.  Integer results against the oracle on the whole batch; H, Hq/Hs
+    and Y (check_rows) on the first, middle and last row of every segment and
+    both sides of every 128-row tile boundary, from each slot's source row;
+    the whole output against the oracle's combine of the GPU's Y."""
+    from test_gpu_swiglu import segment_sample
+    cfg = LAYER8
+    n = cfg.n
+    inp = _spread_scales(workloads.make_inputs(cfg, seed=42, n=n), seed=43)
+    inp_np = parity.numpy_inputs(inp)
+    ref = oracle.run_path(cfg, inp_np, with_recv=False)
+    _, _, b = run_fp8_gpu(cfg, inp, n, fused=True)
+    for key in ("topk_idx", "counts", "expert_off", "slot_of"):
+        assert np.array_equal(parity.to_bits(b[key]).astype(np.int64),
+                              np.asarray(ref[key]).astype(np.int64)), key
+    off, cnt = ref["expert_off"], ref["counts"]
+    assert int(cnt.max()) > 128 and int(cnt[cnt > 0].min()) < 128
+    slots = segment_sample(off, cnt, cfg.n_experts)
+    tok = ref["src_of"][slots] // cfg.top_k
+    expert = np.searchsorted(off[:cfg.n_experts], slots, side="right") - 1
+    check_rows(inp_np, b, slots, expert, x_rows=inp_np["x"][tok],
+               x_scale_rows=inp_np["x_scale"][tok])
+    y_bits = parity.to_bits(b["y"])
+    out_ref = oracle.combine(y_bits, "bf16", ref["topk_w"], ref["slot_of"], "bf16")
+    out_abs = oracle.combine_abs(y_bits, "bf16", ref["topk_w"], ref["slot_of"])
+    parity.assert_combine_close(parity.to_bits(b["out"]), out_ref, out_abs, "bf16")
+
+
 @pytest.mark.parametrize("n,k", [(300, 4), (1000, 8)])
 def test_fp8_swiglu_layer_shape_sampled_rows(n, k):
     """Full D = 7168 and I = 2048 (E = 16 experts to bound the weight bytes):

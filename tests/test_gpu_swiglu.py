@@ -18,17 +18,24 @@ pytestmark = pytest.mark.gpu
 LAYER = workloads.CONFIGS["layer"]
 
 
-def run_layer_gpu(cfg, inp, n):
+def run_layer_gpu(cfg, inp, n, fused=False):
+    """route + dispatch (two calls, or moe_route_dispatch with fused=True) ->
+    grouped SwiGLU GEMMs -> combine on cuda:0."""
     import combine_moe_route_11_b200 as mr
     dev = torch.device("cuda", 0)
     plan = mr.Plan.from_config(cfg, n_max=n)
     ws = plan.new_workspace(dev)
     b = plan.new_buffers(n, dev)
     wgu, wd = inp["w_gate_up"].to(dev), inp["w_down"].to(dev)
-    mr.moe_route_topk(plan, inp["logits"].to(dev), b["topk_idx"], b["topk_w"], b["counts"],
-                      b["expert_off"], ws)
-    mr.moe_dispatch(plan, inp["x"].to(dev), None, b["topk_idx"], b["recv"], None, b["slot_of"],
-                    b["src_of"], ws)
+    logits, x = inp["logits"].to(dev), inp["x"].to(dev)
+    if fused:
+        mr.moe_route_dispatch(plan, logits, x, None, b["topk_idx"], b["topk_w"], b["counts"],
+                              b["expert_off"], b["recv"], None, b["slot_of"], b["src_of"], ws)
+    else:
+        mr.moe_route_topk(plan, logits, b["topk_idx"], b["topk_w"], b["counts"],
+                          b["expert_off"], ws)
+        mr.moe_dispatch(plan, x, None, b["topk_idx"], b["recv"], None, b["slot_of"],
+                        b["src_of"], ws)
     mr.moe_expert_swiglu(plan, n, b["recv"], b["counts"], b["expert_off"], wgu, wd, b["h"],
                          b["y"], ws)
     mr.moe_combine(plan, b["y"], b["topk_w"], b["slot_of"], b["out"], ws)
@@ -63,6 +70,51 @@ def test_swiglu_small_matches_oracle(name, cfg, n):
     parity.assert_layer_out_close(parity.to_bits(b["out"]), ref)
 
 
+def segment_sample(off, cnt, n_experts):
+    """Slots of the first, middle and last row of every expert segment and of
+    the rows on each side of every 128-row tile boundary inside it."""
+    slots = []
+    for e in range(n_experts):
+        if cnt[e]:
+            slots += [off[e], off[e] + cnt[e] - 1, off[e] + cnt[e] // 2]
+            for edge in range(128, int(cnt[e]), 128):
+                slots += [off[e] + edge - 1, off[e] + edge]
+    return np.unique(np.array(slots, np.int64))
+
+
+def test_swiglu_layer_config():
+    """The layer workload exactly as configured and benchmarked: N = 1024,
+    D = 7168, E = 64, k = 8, R = 8, I = 2048, route and dispatch in one launch
+    (moe_route_dispatch, as moe_layer and the bench call it).  About 128 rows
+    per expert, so segments end just below, at or just above a 128-row tile.
+    Integer results are compared with the oracle on the whole batch; Y on the
+    sampled rows of every segment (segment_sample) from each slot's source
+    row; the whole output against the oracle's combine of the GPU's Y."""
+    cfg = LAYER
+    n = cfg.n
+    inp = workloads.make_inputs(cfg, seed=41, n=n)
+    inp_np = parity.numpy_inputs(inp)
+    ref = oracle.run_path(cfg, inp_np, with_recv=False)
+    _, _, b = run_layer_gpu(cfg, inp, n, fused=True)
+    for key in ("topk_idx", "counts", "expert_off", "slot_of"):
+        assert np.array_equal(parity.to_bits(b[key]).astype(np.int64),
+                              np.asarray(ref[key]).astype(np.int64)), key
+    parity.assert_weights_close(parity.to_bits(b["topk_w"]), ref["topk_w"])
+    off, cnt = ref["expert_off"], ref["counts"]
+    assert int(cnt.max()) > 128 and int(cnt[cnt > 0].min()) < 128
+    slots = segment_sample(off, cnt, cfg.n_experts)
+    tok = ref["src_of"][slots] // cfg.top_k
+    expert = np.searchsorted(off[:cfg.n_experts], slots, side="right") - 1
+    rows = np.arange(len(slots), dtype=np.int32)
+    y_ref = oracle.swiglu_rows(rows, expert.astype(np.int32), inp_np["x"][tok],
+                               inp_np["w_gate_up"], inp_np["w_down"])
+    y_bits = parity.to_bits(b["y"])
+    parity.assert_gemm_rows_close(y_bits[slots], y_ref, "Y")
+    out_ref = oracle.combine(y_bits, "bf16", ref["topk_w"], ref["slot_of"], "bf16")
+    out_abs = oracle.combine_abs(y_bits, "bf16", ref["topk_w"], ref["slot_of"])
+    parity.assert_combine_close(parity.to_bits(b["out"]), out_ref, out_abs, "bf16")
+
+
 @pytest.mark.parametrize("n,k", [(300, 4), (1000, 8)])
 def test_swiglu_layer_shape_sampled_rows(n, k):
     """Full D = 7168 and I = 2048 (E = 16 experts to bound the weight bytes):
@@ -77,13 +129,7 @@ def test_swiglu_layer_shape_sampled_rows(n, k):
     off = b["expert_off"].cpu().numpy()
     cnt = b["counts"].cpu().numpy()
     src = b["src_of"].cpu().numpy()
-    slots = []
-    for e in range(cfg.n_experts):
-        if cnt[e]:
-            slots += [off[e], off[e] + cnt[e] - 1, off[e] + cnt[e] // 2]
-            for edge in range(128, int(cnt[e]), 128):
-                slots += [off[e] + edge - 1, off[e] + edge]
-    slots = np.unique(np.array(slots, np.int64))
+    slots = segment_sample(off, cnt, cfg.n_experts)
     tok = src[slots] // cfg.top_k
     expert = np.searchsorted(off[:cfg.n_experts], slots, side="right") - 1
     x_rows = workloads.as_numpy_bits(inp["x"])[tok]
