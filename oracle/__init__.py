@@ -43,6 +43,7 @@ def _sigs():
     i64, i32, ci = ctypes.c_int64, ctypes.c_int32, ctypes.c_int
     return {
         "oracle_route": (ci, [i64, i32, i32, P, P, P]),
+        "oracle_router_logits": (ci, [i64, i32, i32, P, P, P]),
         "oracle_counts": (ci, [i64, i32, i32, P, P]),
         "oracle_region_rows": (i64, [i64, i32, i32, i32]),
         "oracle_offsets": (ci, [i64, i32, i32, i32, P, P]),
@@ -104,6 +105,18 @@ class Oracle:
         w = np.empty((n, top_k), np.float32)
         _check(self.lib.oracle_route(n, e, top_k, _p(logits), _p(idx), _p(w)), "route")
         return idx, w
+
+    def router_logits(self, x: np.ndarray, w_router: np.ndarray) -> np.ndarray:
+        """logits[t, e] = x[t] . w_router[e] over bf16 bits, summed in double,
+        rounded to fp32 ([n, D] and [E, D] uint16 -> [n, E] float32)."""
+        x = np.ascontiguousarray(x, np.uint16)
+        w = np.ascontiguousarray(w_router, np.uint16)
+        n, d = x.shape
+        e, d2 = w.shape
+        assert d == d2, "x and the router weights disagree on D"
+        out = np.empty((n, e), np.float32)
+        _check(self.lib.oracle_router_logits(n, d, e, _p(x), _p(w), _p(out)), "router_logits")
+        return out
 
     def counts(self, topk_idx: np.ndarray, n_experts: int) -> np.ndarray:
         topk_idx = np.ascontiguousarray(topk_idx, dtype=np.int32)

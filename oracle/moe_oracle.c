@@ -8,6 +8,8 @@
  *
  * What it computes, step by step, and the passage each step follows:
  *
+ *   router    logits = x W_r^T per token (bf16 rows and router weights,
+ *             summed in double, rounded to fp32): the gate ahead of top-k.
  *   route     top-k experts per token, ties to the lower expert id, and the
  *             gate weights as a softmax over the k selected logits.  The pages
  *             only fix the shape of the selection ([N, top_k] expert indices,
@@ -152,6 +154,28 @@ int oracle_route(int64_t n, int32_t n_experts, int32_t top_k, const float* logit
         for (int32_t j = 0; j < top_k; ++j) denom += exp(sel[j] - sel[0]);
         for (int32_t j = 0; j < top_k; ++j)
             topk_w[t * top_k + j] = (float)(exp(sel[j] - sel[0]) / denom);
+    }
+    return ORACLE_OK;
+}
+
+/* Router logits: logits[t, e] = sum_d x[t, d] * w_router[e, d] -- the gate
+ * that produces the [N, top_k] expert indices of "backends/mlx: runtime MoE
+ * expert-sort for decode" (author updates on the sorted path) is a linear
+ * map of the token's hidden row; the pages do not spell it out, so the
+ * reading is the plain dot product of the bf16 row with each expert's bf16
+ * router row, summed in double in increasing d and rounded once to fp32.
+ * oracle_route then selects the top k of these logits. */
+int oracle_router_logits(int64_t n, int32_t hidden, int32_t n_experts, const uint16_t* x,
+                         const uint16_t* w_router, float* logits) {
+    if (n < 0 || hidden <= 0 || n_experts <= 0) return ORACLE_BAD_ARG;
+    for (int64_t t = 0; t < n; ++t) {
+        const uint16_t* xr = x + t * hidden;
+        for (int32_t e = 0; e < n_experts; ++e) {
+            const uint16_t* wr = w_router + (int64_t)e * hidden;
+            double acc = 0.0;
+            for (int32_t d = 0; d < hidden; ++d) acc += bf16_to_double(xr[d]) * bf16_to_double(wr[d]);
+            logits[t * n_experts + e] = (float)acc;
+        }
     }
     return ORACLE_OK;
 }

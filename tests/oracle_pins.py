@@ -29,6 +29,46 @@ def _tie_free_logits(n, e, seed=0):
     return (base * 0.37 + r.uniform(-0.1, 0.1, (n, e))).astype(np.float32)
 
 
+# ------------------------------------------------------------------ router
+def _bf16_of(a: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(torch.bfloat16) \
+        .view(torch.int16).numpy().view(np.uint16)
+
+
+def _bf16_f64(b: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).view(torch.bfloat16) \
+        .double().numpy()
+
+
+def pin_router_logits_exact_integers(o):
+    """Small integer-valued bf16 operands make every product and partial sum
+    exact: the logits equal numpy's integer matmul (library) bit for bit,
+    on shapes where E != D so that a transposed operand cannot pass."""
+    r = _rng(11)
+    for (n, d, e) in [(5, 96, 8), (17, 256, 64), (3, 1024, 256)]:
+        xi = r.integers(-8, 9, (n, d))
+        wi = r.integers(-8, 9, (e, d))
+        got = o.router_logits(_bf16_of(xi), _bf16_of(wi))
+        assert np.array_equal(got, (xi @ wi.T).astype(np.float32)), (n, d, e)
+
+
+def pin_router_logits_matmul(o):
+    """Gaussian operands at the router's sizes: the logits are numpy's float64
+    matmul (library) of the decoded bf16 operands rounded to fp32 -- equal
+    except where the two double sums straddle an fp32 rounding point, and
+    never more than one fp32 ulp apart."""
+    r = _rng(12)
+    for (n, d, e) in [(32, 7168, 64), (16, 4096, 128)]:
+        xb = _bf16_of(r.standard_normal((n, d)))
+        wb = _bf16_of(r.standard_normal((e, d)) * 0.02)
+        got = o.router_logits(xb, wb).astype(np.float64)
+        ref64 = _bf16_f64(xb) @ _bf16_f64(wb).T
+        ref = ref64.astype(np.float32).astype(np.float64)
+        ulp = np.spacing(np.abs(ref).astype(np.float32)).astype(np.float64)
+        assert np.all(np.abs(got - ref) <= ulp), (n, d, e)
+        assert np.mean(got == ref) > 0.99, (n, d, e)
+
+
 # ------------------------------------------------------------------ route
 def pin_route_bruteforce(o):
     """Top-k = first k of the full sort of (-logit, id): brute force, with ties."""

@@ -62,6 +62,15 @@ MUTANTS = {
     "fp8_down_h_scale_block": ("(double)hsr[d / block]", "(double)hsr[0]"),
     "fp8_down_expert_scales": ("const float* wsc = w_down_s + e * (int64_t)rb * kb;",
                                "const float* wsc = w_down_s;"),
+    "router_first_expert_row": ("const uint16_t* wr = w_router + (int64_t)e * hidden;",
+                                "const uint16_t* wr = w_router;"),
+    "router_dropped_last_term": ("for (int32_t d = 0; d < hidden; ++d) acc += bf16_to_double(xr[d])",
+                                 "for (int32_t d = 0; d < hidden - 1; ++d) acc += bf16_to_double(xr[d])"),
+    "router_float_accumulator": ("            double acc = 0.0;\n"
+                                 "            for (int32_t d = 0; d < hidden; ++d) acc +=",
+                                 "            float acc = 0.0f;\n"
+                                 "            for (int32_t d = 0; d < hidden; ++d) acc += (float)"),
+    "router_token_row": ("const uint16_t* xr = x + t * hidden;", "const uint16_t* xr = x;"),
 }
 
 
