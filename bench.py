@@ -84,7 +84,8 @@ def describe(cfg, n: int) -> str:
     return s
 
 
-def step_config(cfg, n: int, n_sets: int, world: int, graph: bool = False) -> dict:
+def step_config(cfg, n: int, n_sets: int, world: int, graph: bool = False,
+                two_kernel: bool = False) -> dict:
     """The `config` object shared by both arms' JSON lines."""
     step_bytes = algorithmic_bytes(cfg, n)["step"]
     return {"workload": describe(cfg, n), "parallelism": f"replicas{world}",
@@ -92,7 +93,9 @@ def step_config(cfg, n: int, n_sets: int, world: int, graph: bool = False) -> di
             "l2": (f"no flush: {n_sets} buffer set(s) rotate so a step's data was last touched "
                    f">= 4x L2 ({step_bytes * max(1, n_sets - 1) / 1e6:.0f} MB of traffic) "
                    f"earlier; steps run back to back"),
-            "timed": ("moe_route_dispatch (route: top-k + counts + scan, then dispatch) + "
+            "timed": ("moe_route_topk + moe_dispatch + moe_combine: 3 launches/step"
+                      if two_kernel else
+                      "moe_route_dispatch (route: top-k + counts + scan, then dispatch) + "
                       "moe_combine: " + ("2 launches/step (route and dispatch fused)"
                                          if n <= FUSED_MAX_TOKENS else "3 launches/step")),
             "y_source": "identity expert output, produced once before timing"}
@@ -681,7 +684,7 @@ def run_ours(args, cfg):
     # The step is what moe_route_dispatch + moe_combine launch: one fused
     # route + dispatch kernel for small batches, else the route and dispatch
     # kernels (the very launches moe_route_dispatch makes at that size).
-    if n <= mr.FUSED_MAX_TOKENS:
+    if n <= mr.FUSED_MAX_TOKENS and not args.two_kernel:
         stages = [("route_dispatch", route_dispatch), ("combine", combine)]
     else:
         stages = [("route", route), ("dispatch", dispatch), ("combine", combine)]
@@ -776,7 +779,7 @@ def run_ours(args, cfg):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": path_dtype(cfg), "data": "synthetic",
-            "config": step_config(cfg, n, n_sets, world, args.graph),
+            "config": step_config(cfg, n, n_sets, world, args.graph, args.two_kernel),
             "repeats": len(region_ms),
             "region_ms_per_step": percentiles([r / args.steps for r in region_ms]),
             "step_ms": dict(percentiles(per_step), how="one event after every step"),
@@ -958,6 +961,88 @@ def run_layer(args, cfg):
         dist.destroy_process_group()
 
 
+def run_router(args, cfg):
+    """The router GEMM with the top-k fused (moe_router_topk) on the
+    workload's routing shape: bf16 hidden rows x [N, D] (drawn ~N(0,1)) and
+    router weights [E, D] (~N(0, 0.02)), one call per step (the GEMM with
+    the top-k epilogue, then the counts / offsets kernel).  The roofline
+    line is the call against whichever of the tensor peak (2 N E D flops)
+    and the HBM peak (x and the weights read once, the picks and maps
+    written) needs longer."""
+    world, rank, local = init_dist()
+    import combine_moe_route_11_b200 as mr
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    n, E, D, k = cfg.n, cfg.n_experts, cfg.hidden, cfg.top_k
+    rcfg = cfg.replace(x_dtype="bf16", y_dtype="bf16", out_dtype="bf16", scale_block=0)
+    plan = mr.Plan.from_config(rcfg, n_max=n)
+    gen = torch.Generator(device=dev).manual_seed(2000 + rank)
+    # enough buffer sets that a set's x was last read >= 4x L2 earlier
+    x_bytes = n * D * 2
+    n_sets = max(1, min(16, -(-4 * L2_BYTES // x_bytes) + 1)) if x_bytes < 4 * L2_BYTES else 1
+    xs = [torch.randn(n, D, generator=gen, device=dev).to(torch.bfloat16) for _ in range(n_sets)]
+    w = (torch.randn(E, D, generator=gen, device=dev) * 0.02).to(torch.bfloat16)
+    ws = plan.new_workspace(dev)
+    b = plan.new_buffers(n, dev)
+
+    def step(i):
+        mr.moe_router_topk(plan, xs[i % n_sets], w, None, b["topk_idx"], b["topk_w"],
+                           b["counts"], b["expert_off"], ws, stream)
+
+    for i in range(args.warmup):
+        step(i)
+    sampler = ClockSampler(local)
+    sampler.wait_first()
+
+    def region():
+        for i in range(args.steps):
+            step(i)
+
+    region_ms, t_start, t_end = timed_regions(region, stream, dev, args.steps)
+    clocks = sampler.stop(t_start, t_end)
+    if mr.moe_get_status(plan, ws, stream) != 0:
+        raise RuntimeError("device status set during timing")
+    ms_step = statistics.median(region_ms) / args.steps
+    flops = 2.0 * n * E * D
+    nbytes = x_bytes + E * D * 2 + n * k * 8 + n * k * 4 + (2 * E + 1) * 4
+    t = ms_step * 1e-3
+    peaks = {}
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peaks = json.load(f)
+    except OSError:
+        pass
+    tpeak = float(peaks.get("bf16_tflops", 1590.0))
+    hpeak, hkind = read_peaks()
+    tensor_line = {"bound": "tensor", "kernel": "moe_router_topk (router GEMM + top-k, counts)",
+                   "achieved": flops / t / 1e12, "peak": tpeak,
+                   "peak_kind": "measured burst" if peaks else "fallback",
+                   "unit": "TFLOP/s", "frac": flops / t / 1e12 / tpeak, "traffic": None}
+    hbm_line = {"bound": "hbm", "kernel": "moe_router_topk (router GEMM + top-k, counts)",
+                "achieved": nbytes / t / 1e9, "peak": hpeak, "peak_kind": hkind, "unit": "GB/s",
+                "frac": nbytes / t / 1e9 / hpeak, "traffic": None, "algorithmic_bytes": nbytes}
+    hbm_bound = nbytes / (hpeak * 1e9) >= flops / (tpeak * 1e12)
+    roofline, other = (hbm_line, tensor_line) if hbm_bound else (tensor_line, hbm_line)
+    if rank == 0:
+        print(json.dumps({
+            "metric": "router GEMM + top-k tokens/s (moe_router_topk)",
+            "value": world * n / t, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16 hidden rows and router weights, fp32 accumulate and logits",
+            "data": "synthetic (x ~ N(0,1), router weights ~ N(0, 0.02), drawn on the device)",
+            "config": {"workload": f"{cfg.name} routing shape: N={n}, D={D}, E={E}, k={k}, "
+                                   f"R={cfg.n_ranks}, bf16 hidden rows",
+                       "l2": f"{n_sets} x buffer set(s) rotate"},
+            "repeats": len(region_ms),
+            "region_ms_per_step": percentiles([r / args.steps for r in region_ms]),
+            "roofline": roofline, "roofline_other": other,
+            "gpu_launches": 2 * args.steps, "clocks": clocks}), flush=True)
+    if dist.is_available() and dist.is_initialized():
+        dist.destroy_process_group()
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -967,6 +1052,12 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--router", action="store_true",
+                    help="time the router GEMM with the top-k fused (moe_router_topk) on the "
+                         "workload's routing shape instead")
+    ap.add_argument("--two-kernel", action="store_true",
+                    help="time the route and dispatch kernels (moe_route_topk + moe_dispatch) "
+                         "even where moe_route_dispatch would run them as one launch")
     ap.add_argument("--graph", action="store_true",
                     help="replay each step as one captured CUDA graph")
     ap.add_argument("--tokens", type=int, default=0,
@@ -983,9 +1074,11 @@ def main(argv=None):
     if args.experts:
         cfg = cfg.replace(n_experts=args.experts)
     if args.impl == "reference":
-        if cfg.inter > 0:
+        if cfg.inter > 0 or args.router:
             ap.error("the reference arm times the identity-expert path")
         run_reference(args, cfg)
+    elif args.router:
+        run_router(args, cfg)
     elif cfg.inter > 0:
         run_layer(args, cfg)
     else:

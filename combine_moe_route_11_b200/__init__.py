@@ -14,7 +14,8 @@ import os
 import torch
 
 __all__ = [
-    "MoeError", "Plan", "LIB_PATH", "moe_route_topk", "moe_dispatch", "moe_route_dispatch",
+    "MoeError", "Plan", "LIB_PATH", "moe_route_topk", "moe_router_topk", "moe_dispatch",
+    "moe_route_dispatch",
     "moe_expert_dequant", "moe_expert_swiglu", "moe_expert_swiglu_fp8", "moe_combine",
     "moe_layer", "moe_layer_fp8", "moe_layer_buffer",
     "moe_get_status", "moe_workspace_init", "moe_strerror", "DTYPE_CODES", "ELEM_BYTES",
@@ -53,6 +54,7 @@ _SIGS = {
     "moe_region_rows": (ctypes.c_int64, [_P, _i32]),
     "moe_recv_rows": (ctypes.c_int64, [_P, _i32]),
     "moe_route_topk": (ctypes.c_int, [_P, _i32, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_router_topk": (ctypes.c_int, [_P, _i32, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_dispatch": (ctypes.c_int, [_P, _i32, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_route_dispatch": (ctypes.c_int, [_P, _i32] + [_P] * 13),
     "moe_expert_dequant": (ctypes.c_int, [_P, _i32, _P, _P, _P, _P, _P, _P]),
@@ -245,6 +247,24 @@ def moe_route_topk(plan: Plan, logits, topk_idx, topk_w, counts, expert_off, ws,
     _check(_lib.moe_route_topk(plan.handle, n, _ptr(logits), _ptr(topk_idx), _ptr(topk_w),
                                _ptr(counts), _ptr(expert_off), _ws(plan, ws), _stream(stream)),
            "moe_route_topk")
+
+
+def moe_router_topk(plan: Plan, x, w_router, logits, topk_idx, topk_w, counts, expert_off, ws,
+                    stream=None):
+    """Router GEMM (logits = x w_router^T) with top-k and softmax fused, then
+    counts and offsets; x is the bf16 [n, D] hidden rows, logits may be None."""
+    n = x.shape[0]
+    _expect(x, (torch.bfloat16,), (n, plan.hidden), "x")
+    _expect(w_router, (torch.bfloat16,), (plan.n_experts, plan.hidden), "w_router")
+    if logits is not None:
+        _expect(logits, (torch.float32,), (n, plan.n_experts), "logits")
+    _expect(topk_idx, (torch.int32,), (n, plan.top_k), "topk_idx")
+    _expect(topk_w, (torch.float32,), (n, plan.top_k), "topk_w")
+    _expect(counts, (torch.int32,), (plan.n_experts,), "counts")
+    _expect(expert_off, (torch.int32,), (plan.n_experts + 1,), "expert_off")
+    _check(_lib.moe_router_topk(plan.handle, n, _ptr(x), _ptr(w_router), _ptr(logits),
+                                _ptr(topk_idx), _ptr(topk_w), _ptr(counts), _ptr(expert_off),
+                                _ws(plan, ws), _stream(stream)), "moe_router_topk")
 
 
 def _check_dispatch_outputs(plan: Plan, T: int, x_scale, n: int, recv, recv_scale, slot_of,

@@ -19,9 +19,8 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmoeroute.so")
 OBJ_DIR = os.path.join(PKG, "_build")
 
-SOURCES = ["api.cu", "route.cu", "route_dispatch.cu", "dispatch.cu", "combine.cu", "swiglu_gemm.cu",
-           "fp8_gemm.cu",
-           "route_noalloc.cu"]
+SOURCES = ["api.cu", "route.cu", "router_gemm.cu", "route_dispatch.cu", "dispatch.cu", "combine.cu",
+           "swiglu_gemm.cu", "fp8_gemm.cu", "route_noalloc.cu"]
 HEADERS = ["moe_internal.cuh", "route_common.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",

@@ -1,7 +1,7 @@
 // C ABI of libmoeroute: plan validation, workspace layout and the entry
 // points declared in include/moeroute.h.  Host code only; every step of the
-// path runs in the kernels of route.cu, route_dispatch.cu, dispatch.cu,
-// combine.cu, swiglu_gemm.cu, fp8_gemm.cu and route_noalloc.cu.  The per-device caches
+// path runs in the kernels of route.cu, router_gemm.cu, route_dispatch.cu,
+// dispatch.cu, combine.cu, swiglu_gemm.cu, fp8_gemm.cu and route_noalloc.cu.  The per-device caches
 // here and in the launchers may be reached from several host threads.
 #include "moe_internal.cuh"
 
@@ -64,14 +64,14 @@ Layout make_layout(const moe_plan& p) {
     return here;
   };
   L.ctrl = take(sizeof(Ctrl));
-  // right after ctrl, all cleared together by moe_workspace_init: expert totals
-  // [2, E] and token masks [2, mask rows, E], each double-buffered by the
-  // grid-barrier generation
-  L.totals = take(size_t(2) * d.n_experts * 4);
+  // right after ctrl, all cleared together by moe_workspace_init: the route
+  // kernel's look-back words [2, route blocks, E] (alternate halves per call)
+  // and the fused kernel's token masks [2, mask rows, E] (alternate halves by
+  // its grid-barrier generation)
+  L.flags = take(size_t(2) * p.blocks_max * d.n_experts * 4);
   L.masks = take(size_t(2) * mask_rows(p) * d.n_experts * 4);
-  L.blk = take(size_t(p.blocks_max) * d.n_experts * 4);
-  L.bases = take(size_t(p.blocks_max) * d.n_experts * 4);
-  L.rank = take(size_t(d.n_max) * d.top_k);
+  L.pos = take(size_t(d.n_max) * d.top_k * 4);
+  L.off = take(size_t(d.n_experts + 1) * 4);
   L.route_end = at;
   const size_t nk = size_t(d.n_max) * d.top_k;
   const size_t T = size_t(p.total_max);
@@ -117,6 +117,8 @@ moe_status moe_plan_create(const moe_desc* desc, moe_plan** out) {
   const moe_desc d = *desc;
   if (d.n_max < 1 || d.hidden < 1 || d.n_experts < 1 || d.top_k < 1 || d.n_ranks < 1)
     return MOE_ERR_INVALID_ARG;
+  // per-expert counts travel in 30-bit fields of the route kernel's look-back words
+  if (d.n_max >= (1 << 30)) return MOE_ERR_UNSUPPORTED;
   if (d.n_experts > kMaxExperts || d.top_k > kMaxTopK) return MOE_ERR_UNSUPPORTED;
   if (d.top_k > d.n_experts || d.n_experts % d.n_ranks != 0) return MOE_ERR_INVALID_ARG;
   auto dtype_ok = [](int t) { return t == MOE_F32 || t == MOE_BF16 || t == MOE_FP8_E4M3; };
@@ -182,6 +184,21 @@ moe_status moe_route_topk(const moe_plan* p, int32_t n, const float* logits, int
                                   reinterpret_cast<cudaStream_t>(stream)));
 }
 
+moe_status moe_router_topk(const moe_plan* p, int32_t n, const void* x, const void* w_router,
+                           float* logits, int32_t* topk_idx, float* topk_w, int32_t* counts,
+                           int32_t* expert_off, void* ws, moe_stream_t stream) {
+  moe_status s = check_call(p, n, ws);
+  if (s != MOE_OK) return s;
+  if (p->d.hidden % 64 != 0 || p->d.n_experts > 256) return MOE_ERR_UNSUPPORTED;
+  if (!counts || !expert_off || (n > 0 && (!x || !w_router || !topk_idx || !topk_w)))
+    return MOE_ERR_INVALID_ARG;
+  if (n > 0 && (!aligned16(x) || !aligned16(w_router))) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  s = cuda_status(launch_router(*p, n, x, w_router, logits, topk_idx, topk_w, ws, st));
+  if (s != MOE_OK) return s;
+  return cuda_status(launch_route_counts(*p, n, topk_idx, counts, expert_off, ws, st));
+}
+
 moe_status moe_dispatch(const moe_plan* p, int32_t n, const void* x, const float* x_scale,
                         const int32_t* topk_idx, void* recv, float* recv_scale, int32_t* slot_of,
                         int32_t* src_of, void* ws, moe_stream_t stream) {
@@ -191,6 +208,8 @@ moe_status moe_dispatch(const moe_plan* p, int32_t n, const void* x, const float
   if (!x || !topk_idx || !recv || !slot_of || !src_of) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(recv)) return MOE_ERR_INVALID_ARG;
   if (p->scale_cols > 0 && (!x_scale || !recv_scale)) return MOE_ERR_INVALID_ARG;
+  if (p->scale_cols > 0 && (!aligned16(x_scale) || !aligned16(recv_scale)))
+    return MOE_ERR_INVALID_ARG;
   return cuda_status(launch_dispatch(*p, n, x, x_scale, topk_idx, recv, recv_scale, slot_of,
                                      src_of, ws, reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -207,6 +226,8 @@ moe_status moe_route_dispatch(const moe_plan* p, int32_t n, const float* logits,
       return MOE_ERR_INVALID_ARG;
     if (!aligned16(logits) || !aligned16(x) || !aligned16(recv)) return MOE_ERR_INVALID_ARG;
     if (p->scale_cols > 0 && (!x_scale || !recv_scale)) return MOE_ERR_INVALID_ARG;
+    if (p->scale_cols > 0 && (!aligned16(x_scale) || !aligned16(recv_scale)))
+      return MOE_ERR_INVALID_ARG;
   }
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (route_blocks(n) <= kFusedMaxBlocks)
@@ -320,7 +341,7 @@ moe_status layer_impl(const moe_plan* p, int32_t n, const float* logits, const v
   if (n > 0) {
     if (!logits || !x || !out) return MOE_ERR_INVALID_ARG;
     if (!aligned16(logits) || !aligned16(x) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
-    if (p->scale_cols > 0 && !x_scale) return MOE_ERR_INVALID_ARG;
+    if (p->scale_cols > 0 && (!x_scale || !aligned16(x_scale))) return MOE_ERR_INVALID_ARG;
     if (d.inter > 0 && (!aligned16(w_gate_up) || !aligned16(w_down))) return MOE_ERR_INVALID_ARG;
   }
   char* b = static_cast<char*>(ws);
@@ -391,8 +412,8 @@ moe_status moe_get_status(const moe_plan* p, void* ws, moe_stream_t stream) {
 
 moe_status moe_workspace_init(const moe_plan* p, void* ws, moe_stream_t stream) {
   if (!p || !ws) return MOE_ERR_INVALID_ARG;
-  // control words, expert totals and token masks (which follow them)
-  return cudaMemsetAsync(ws, 0, p->lay.blk, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+  // control words, look-back words and token masks (which follow them)
+  return cudaMemsetAsync(ws, 0, p->lay.pos, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
              ? MOE_OK
              : MOE_ERR_CUDA;
 }

@@ -9,8 +9,9 @@
 // divides both the 7168-byte FP8 rows and the 14336-byte bf16 rows of the
 // workloads, and 32 registers per thread let 8 blocks share an SM.  Every
 // lane loads 2 sixteen-byte vectors of the chunk first (they do not depend on
-// routing), while lanes j < k resolve the slot of choice j -- the route
-// call's per-block base plus the in-block rank, no metadata round trip --
+// routing), while lanes j < k resolve the slot of choice j -- the expert's
+// offset plus the pick's in-expert position, both left in the workspace by
+// the route call, no metadata round trip --
 // then the warp stores the chunk k times.  Scales and the index maps go with
 // the first chunk of the row.  High occupancy keeps enough loads and stores
 // in flight: on B200 this beats staging the chunks through shared memory
@@ -30,8 +31,8 @@ struct DispatchArgs {
   const uint8_t* x;
   const float* x_scale;
   const int32_t* topk_idx;
-  const int32_t* bases;  // per-(route block, expert) base slot
-  const uint8_t* rank;   // [n, k] in-block rank
+  const int32_t* off;    // [E + 1] expert offsets (the route call's copy)
+  const int32_t* pos;    // [n, k] position of each pick inside its expert's segment
   uint8_t* recv;
   float* recv_scale;
   int32_t* slot_of;
@@ -65,7 +66,7 @@ __global__ void __launch_bounds__(kThreads, 8) dispatch_kernel(DispatchArgs a) {
       const int64_t tk = t * a.K + lane;
       const int e = __ldg(a.topk_idx + tk);
       if (e >= 0 && e < a.E) {
-        slot = __ldg(a.bases + (t / kRouteTokens) * a.E + e) + a.rank[tk];
+        slot = __ldg(a.off + e) + __ldg(a.pos + tk);
         if (slot < 0 || slot >= a.total) slot = -1;
       }
       if (slot < 0) set_status(a.ws, MOE_ERR_DEVICE_INDEX);
@@ -85,12 +86,25 @@ __global__ void __launch_bounds__(kThreads, 8) dispatch_kernel(DispatchArgs a) {
       }
     }
     if (c == 0 && a.S > 0) {
-      for (int i0 = 0; i0 < a.S; i0 += 32) {
-        const int i = i0 + lane;
-        const float sv = i < a.S ? __ldcs(a.x_scale + t * a.S + i) : 0.f;
+      if ((a.S & 3) == 0 && a.S <= 128) {
+        // the row's scales as 16-byte vectors, one per lane (a single store
+        // instruction per copy for the 56 scales of a 7168-column row)
+        const int nv = a.S >> 2;
+        float4 sv = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (lane < nv) sv = __ldcs(reinterpret_cast<const float4*>(a.x_scale + t * a.S) + lane);
         for (int j = 0; j < a.K; ++j) {
           const int s = __shfl_sync(0xFFFFFFFFu, slot, j);
-          if (s >= 0 && i < a.S) __stcs(a.recv_scale + int64_t(s) * a.S + i, sv);
+          if (s >= 0 && lane < nv)
+            __stcs(reinterpret_cast<float4*>(a.recv_scale + int64_t(s) * a.S) + lane, sv);
+        }
+      } else {
+        for (int i0 = 0; i0 < a.S; i0 += 32) {
+          const int i = i0 + lane;
+          const float sv = i < a.S ? __ldcs(a.x_scale + t * a.S + i) : 0.f;
+          for (int j = 0; j < a.K; ++j) {
+            const int s = __shfl_sync(0xFFFFFFFFu, slot, j);
+            if (s >= 0 && i < a.S) __stcs(a.recv_scale + int64_t(s) * a.S + i, sv);
+          }
         }
       }
     }
@@ -108,8 +122,8 @@ cudaError_t launch_dispatch(const moe_plan& p, int32_t n, const void* x, const f
   a.x = static_cast<const uint8_t*>(x);
   a.x_scale = x_scale;
   a.topk_idx = topk_idx;
-  a.bases = reinterpret_cast<const int32_t*>(static_cast<const char*>(ws) + p.lay.bases);
-  a.rank = reinterpret_cast<const uint8_t*>(static_cast<const char*>(ws) + p.lay.rank);
+  a.off = reinterpret_cast<const int32_t*>(static_cast<const char*>(ws) + p.lay.off);
+  a.pos = reinterpret_cast<const int32_t*>(static_cast<const char*>(ws) + p.lay.pos);
   a.recv = static_cast<uint8_t*>(recv);
   a.recv_scale = recv_scale;
   a.slot_of = slot_of;

@@ -131,20 +131,33 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
-// 16 consecutive fp32 columns of this thread's TMEM lane (16 rather than 32
-// temporaries keep the 128 accumulators of a thread inside the register budget).
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
-  uint32_t r[16];
+// 8 consecutive fp32 columns of this thread's TMEM lane.  The 128
+// accumulators of a promotion thread and the temporaries of one load must fit
+// in 168 registers: 320 threads put three warps on one of the SM's four
+// register-file partitions of 16 K registers, so no thread may have more.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+  uint32_t r[8];
   asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
-      "%12, %13, %14, %15}, [%16];"
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15])
+        "=r"(r[7])
       : "r"(taddr));
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// The per-k-block waits of this kernel run about 50 times as often as the
+// bf16 kernel's per-tile waits.  Poll by count first (mbarrier.try_wait
+// already suspends the thread for a while when the phase is not complete)
+// and read the clock only for a wait that lasts; still bounded, by
+// kHotPolls polls plus mbar_wait's clock limit.
+constexpr int kHotPolls = 1024;
+
+__device__ __forceinline__ bool mbar_wait_hot(uint64_t* bar, uint32_t parity) {
+  for (int i = 0; i < kHotPolls; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait(bar, parity);
 }
 
 struct Tile {
@@ -252,15 +265,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t issued_phase[kStages];
-      bool issued[kStages];
-      for (int s = 0; s < kStages; ++s) issued[s] = false, issued_phase[s] = 0;
+      int issued = 0;  // copies issued, in ring order
       for (int t = blockIdx.x; t < total && !*s_abort; t += gridDim.x) {
         const Tile tl = tile_of(t, s_pref, E, g.n_tiles);
         const int a_row = g.expert_off[tl.e] + tl.m * kBM;
         const int b_row = tl.e * g.b_rows + tl.n * (kSwiGLU ? kBN / 2 : kBN);
         for (int kb = 0; kb < g.k_steps; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u)) {
+          if (!mbar_wait_hot(&empty[stage], phase ^ 1u)) {
             set_status(g.ws, MOE_ERR_TIMEOUT);
             *s_abort = 1;
             break;
@@ -275,14 +286,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             tma_load_2d(b_dst, &tma_b, kb * kBK, b_row, &full[stage]);
           }
-          issued[stage] = true;
-          issued_phase[stage] = phase;
+          ++issued;
           if (++stage == kStages) stage = 0, phase ^= 1u;
         }
       }
-      // never leave a copy in flight into this CTA's shared memory
-      for (int s = 0; s < kStages; ++s)
-        if (issued[s] && !mbar_wait(&full[s], issued_phase[s])) set_status(g.ws, MOE_ERR_TIMEOUT);
+      // never leave a copy in flight into this CTA's shared memory: a copy
+      // was only issued into a stage once the MMAs had consumed the copy
+      // before it, so only the last kStages copies can still be unwaited
+      for (int i = issued > kStages ? issued - kStages : 0; i < issued; ++i)
+        if (!mbar_wait(&full[i % kStages], uint32_t(i / kStages) & 1u))
+          set_status(g.ws, MOE_ERR_TIMEOUT);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -293,8 +306,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
         for (int kb = 0; kb < g.k_steps; ++kb) {
-          if (*s_abort || !mbar_wait(&pempty[buf], buf_phase ^ 1u) ||
-              !mbar_wait(&full[stage], phase)) {
+          if (*s_abort || !mbar_wait_hot(&pempty[buf], buf_phase ^ 1u) ||
+              !mbar_wait_hot(&full[stage], phase)) {
             if (!*s_abort) set_status(g.ws, MOE_ERR_TIMEOUT);
             *s_abort = 1;
             ok = false;
@@ -332,7 +345,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t row = int64_t(g.expert_off[tl.e]) + tl.m * kBM + r_local;
       // a segment outside [0, T) (caller-supplied counts or offsets) is skipped
       const bool in_range = row >= 0 && row < g.total;
-      const float* sa_row = g.a_scale + (in_range ? row : 0) * g.k_steps;
+      // scale offsets as 32-bit element indices (T * k_steps and
+      // E * b_rows / 128 * k_steps stay far below 2^31): fewer live registers
+      // next to the 128 accumulators
+      const int sa_off = int(in_range ? row : 0) * g.k_steps;
       // scale rows of the weight tiles under chunks 0-1 and 2-3
       int brow0, brow1;
       if (kSwiGLU) {
@@ -341,18 +357,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         brow0 = brow1 = tl.e * b_blocks + 2 * tl.n + half;
       }
-      const float* sb0 = g.b_scale + int64_t(brow0) * g.k_steps;
-      const float* sb1 = g.b_scale + int64_t(brow1) * g.k_steps;
+      const int sb0_off = brow0 * g.k_steps;
+      const int sb1_off = brow1 * g.k_steps;
       float acc[kCols];
 #pragma unroll
       for (int i = 0; i < kCols; ++i) acc[i] = 0.f;
       bool ok = true;
       for (int kb = 0; kb < g.k_steps; ++kb) {
-        const float sa = in_range ? __ldg(sa_row + kb) : 0.f;
-        const float s0 = sa * __ldg(sb0 + kb);
-        const float s1 = sa * __ldg(sb1 + kb);
+        const float sa = in_range ? __ldg(g.a_scale + (sa_off + kb)) : 0.f;
+        const float s0 = sa * __ldg(g.b_scale + (sb0_off + kb));
+        const float s1 = sa * __ldg(g.b_scale + (sb1_off + kb));
         bool ready = true;
-        if (lane == 0) ready = !*s_abort && mbar_wait(&pfull[buf], buf_phase);
+        if (lane == 0) ready = !*s_abort && mbar_wait_hot(&pfull[buf], buf_phase);
         ready = __shfl_sync(0xFFFFFFFFu, ready ? 1 : 0, 0) != 0;
         if (!ready) {
           if (lane == 0 && !*s_abort) set_status(g.ws, MOE_ERR_TIMEOUT);
@@ -366,12 +382,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < 4; ++j) {
           const float sc = (kSwiGLU && j >= 2) ? s1 : s0;
 #pragma unroll
-          for (int hj = 0; hj < 2; ++hj) {
-            float v[16];
-            tmem_ld16(taddr + uint32_t(chunk_col<kSwiGLU>(half, j) + hj * 16), v);
+          for (int hj = 0; hj < 4; ++hj) {
+            float v[8];
+            tmem_ld8(taddr + uint32_t(chunk_col<kSwiGLU>(half, j) + hj * 8), v);
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              acc[j * 32 + hj * 16 + i] = fmaf(v[i], sc, acc[j * 32 + hj * 16 + i]);
+            for (int i = 0; i < 8; ++i)
+              acc[j * 32 + hj * 8 + i] = fmaf(v[i], sc, acc[j * 32 + hj * 8 + i]);
           }
         }
         tc_fence_before();

@@ -1,5 +1,5 @@
 // Route: top-k gating, per-expert counts, rank-major expert offsets and the
-// per-block bases from which moe_dispatch derives every slot.
+// in-expert position of every pick, from which moe_dispatch derives slots.
 //
 // Slots follow the rank-major layout of the one-sided expert-parallel
 // all-to-all ("One-Sided Expert-Parallel All-to-All for Mixture-of-Experts
@@ -10,215 +10,277 @@
 // ("backends/mlx: runtime MoE expert-sort for decode", author update on the
 // sorted branch) -- computed here as a counting sort, without any sort.
 //
-// One cooperative launch (all blocks resident), two phases split by a
-// bounded grid barrier:
-//  1. per route block of 32 tokens, one warp per token: the k largest logits
-//     by k rounds of a warp argmax on order-preserving integer keys (two
-//     single-instruction warp reductions per round; the lower expert id wins
-//     a tie) and a softmax over the k winners; then, per expert, the bitmask
-//     of the block's tokens that picked it gives each (token, expert) pair
-//     its rank among the block's tokens (popcount of the lower lanes) and the
-//     block's count of the expert;
-//     Each block also adds its counts into the expert totals (integer
-//     atomics: the sum does not depend on their order);
-//  2. per column of (up to) 4 experts: the totals of the experts of its rank
-//     below its own give the rank-major offsets, and an exclusive scan of its
-//     own count columns over the route blocks gives each block's absolute
-//     base slot.
-// A slot is then base[block][e] + rank.  All integer results are
-// deterministic: no atomic decides an order.
+// One ordinary launch, one pass, no grid-wide barrier.  A block takes a
+// ticket from a counter in the workspace: ticket b is route block b, tokens
+// [32b, 32b + 32).  Tickets are handed out in the order blocks start, so a
+// block only ever waits on blocks that are already running.
+//  1. One warp per token (several tokens per warp): the k largest logits by
+//     k rounds of a warp argmax on order-preserving integer keys (the lower
+//     expert id wins a tie) and a softmax over the k winners.
+//  2. Per expert, the bitmask of the block's tokens that picked it gives each
+//     pick its rank among the block's tokens (popcount of the lower bits) and
+//     the block's count c[b][e].
+//  3. Decoupled look-back, one thread per expert column: block b publishes
+//     c[b][e] as an aggregate, then sums the published words of blocks
+//     b-1, b-2, ... (a window of loads at a time) until it meets an inclusive
+//     prefix; it then publishes its own inclusive prefix.  Block 0 publishes
+//     an inclusive prefix at once.  Each word is one 32-bit store: a ready
+//     bit, an inclusive bit and the count, so no fence orders value and flag.
+//  4. The position of every pick inside its expert's segment is the block's
+//     exclusive prefix plus the in-block rank.
+//  5. The block holding the last ticket has every expert's total as its
+//     inclusive prefix: it turns them into the rank-major offsets.
+// All integer results are deterministic: no atomic decides an order.
+//
+// The look-back words alternate between two halves of a table in the
+// workspace: a call uses one half, clears the rows of the other half that
+// the previous call wrote, and the last block flips the half for the next
+// call.  Every wait is bounded; a wait that gives up records MOE_ERR_TIMEOUT
+// and the workspace must be re-initialised.
 #include "route_common.cuh"
 
 #include <atomic>
 
-#include <float.h>
-#include <limits.h>
-
-#include <type_traits>
-
 namespace moe {
 namespace {
 
-static_assert(kWarps == 32, "phase 2 scans one sum per warp with one warp");
+constexpr int kLbWarps = 8;                    // warps per route block
+constexpr int kLbThreads = kLbWarps * 32;
+constexpr int kTokPerWarp = kRouteTokens / kLbWarps;
+constexpr int kWindow = 16;                    // look-back words per window
+constexpr int kExpPerThread = (kMaxExperts + kLbThreads - 1) / kLbThreads;
 
-// Phase 2 for column unit u (experts [u*W, u*W + W)): rank-major offsets
-// from the expert totals, then the exclusive scan of the unit's count columns
-// over the route blocks into absolute bases.
-template <int W>
-__device__ __forceinline__ void scan_column(const RouteArgs& a, int u, const int32_t* tot,
-                                            void* s_warp_raw, int32_t* s_off) {
-  using V = typename std::conditional<W == 4, int4, int>::type;
-  V* s_warp = static_cast<V*>(s_warp_raw);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int B = a.blocks, E = a.E;
-  const int per_rank = E / a.R;
-  const int e0 = u * W;
-  const int64_t row = E / W;  // row stride in column units
-  V zero;
-  if constexpr (W == 4) zero = make_int4(0, 0, 0, 0);
-  else zero = 0;
-  auto add = [](V& x, const V& y) {
-    if constexpr (W == 4) { x.x += y.x; x.y += y.y; x.z += y.z; x.w += y.w; }
-    else x += y;
-  };
-  const V* cnt = reinterpret_cast<const V*>(a.blk);
-  // ---- this thread's blocks of the unit's count columns, loaded first: they
-  // do not depend on the offsets below
-  V* base = reinterpret_cast<V*>(a.bases) + u;
-  const V* own = cnt + u;
-  const int per = (B + kRouteThreads - 1) / kRouteThreads;
-  const int b0 = min(B, tid * per), b1 = min(B, b0 + per);
-  V sum = zero;
-  for (int b = b0; b < b1; ++b) add(sum, __ldcg(own + int64_t(b) * row));
-  // ---- offsets of this unit's experts from the phase-1 totals: one warp each
-  if (warp < W) {
-    const int e = e0 + warp;
-    const int r = e / per_rank;
-    int tsum = 0;
-    for (int e2 = r * per_rank + lane; e2 < e; e2 += 32) tsum += __ldcg(tot + e2);
-    tsum = __reduce_add_sync(kFull, tsum);
-    if (lane == 0) {
-      const int off = r * a.region_rows + tsum;
-      s_off[warp] = off;
-      a.expert_off[e] = off;
-      a.counts[e] = __ldcg(tot + e);
-    }
-  }
-  // ---- exclusive scan of the columns over the route blocks: within each
-  // warp, then of the warp sums by warp 0
-  V incl = sum;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    V y;
-    if constexpr (W == 4) {
-      y.x = __shfl_up_sync(kFull, incl.x, o); y.y = __shfl_up_sync(kFull, incl.y, o);
-      y.z = __shfl_up_sync(kFull, incl.z, o); y.w = __shfl_up_sync(kFull, incl.w, o);
-    } else {
-      y = __shfl_up_sync(kFull, incl, o);
-    }
-    if (lane >= o) add(incl, y);
-  }
-  if (lane == 31) s_warp[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    const V w = s_warp[lane];  // kWarps == 32 warp sums
-    V wi = w;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      V y;
-      if constexpr (W == 4) {
-        y.x = __shfl_up_sync(kFull, wi.x, o); y.y = __shfl_up_sync(kFull, wi.y, o);
-        y.z = __shfl_up_sync(kFull, wi.z, o); y.w = __shfl_up_sync(kFull, wi.w, o);
-      } else {
-        y = __shfl_up_sync(kFull, wi, o);
-      }
-      if (lane >= o) add(wi, y);
-    }
-    if constexpr (W == 4) { wi.x -= w.x; wi.y -= w.y; wi.z -= w.z; wi.w -= w.w; }
-    else wi -= w;
-    s_warp[lane] = wi;  // exclusive prefix of the warp sums
-  }
-  __syncthreads();
-  V run;
-  if constexpr (W == 4) run = make_int4(s_off[0], s_off[1], s_off[2], s_off[3]);
-  else run = s_off[0];
-  add(run, s_warp[warp]);
-  // run + (incl - sum) = absolute base of this thread's first block
-  V ex = incl;
-  if constexpr (W == 4) { ex.x -= sum.x; ex.y -= sum.y; ex.z -= sum.z; ex.w -= sum.w; }
-  else ex -= sum;
-  add(run, ex);
-  for (int b = b0; b < b1; ++b) {
-    base[int64_t(b) * row] = run;
-    if (b + 1 < b1) add(run, __ldcg(own + int64_t(b) * row));
-  }
-  __syncthreads();  // shared scratch is reused by the next unit
+constexpr uint32_t kReady = 0x40000000u;
+constexpr uint32_t kIncl = 0x80000000u;
+constexpr uint32_t kValue = 0x3FFFFFFFu;
+
+__device__ __forceinline__ uint32_t ld_relaxed_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
 }
 
-template <int VPL, int VEC>
-__global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(RouteArgs a) {
+__device__ __forceinline__ void st_relaxed_u32(uint32_t* p, uint32_t v) {
+  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// A published look-back word; waits (bounded) until it is ready.  A wait
+// that gives up records MOE_ERR_TIMEOUT and reads as an inclusive zero, so
+// the look-back ends.
+__device__ __forceinline__ uint32_t wait_ready(const uint32_t* p, uint32_t v, void* ws) {
+  if (v & kReady) return v;
+  const long long t0 = clock64();
+  while (!((v = ld_relaxed_gpu(p)) & kReady)) {
+    if (clock64() - t0 > (1ll << 31)) {
+      set_status(ws, MOE_ERR_TIMEOUT);
+      return kReady | kIncl;
+    }
+  }
+  return v;
+}
+
+// Exclusive prefix of column `col` over the route blocks below b: windows of
+// kWindow words, the next window's loads in flight while the current one is
+// summed, until an inclusive prefix turns up.
+__device__ __forceinline__ void load_window(const uint32_t* col, int p, int stride,
+                                            uint32_t (&w)[kWindow]) {
+#pragma unroll
+  for (int i = 0; i < kWindow; ++i)
+    w[i] = p - i >= 0 ? ld_relaxed_gpu(col + int64_t(p - i) * stride) : (kReady | kIncl);
+}
+
+__device__ __forceinline__ int look_back(const uint32_t* col, int b, int stride, void* ws) {
+  int excl = 0;
+  uint32_t cur[kWindow], nxt[kWindow];
+  load_window(col, b - 1, stride, cur);
+  for (int p = b - 1; p >= 0; p -= kWindow) {
+    if (p - kWindow >= 0) load_window(col, p - kWindow, stride, nxt);
+#pragma unroll
+    for (int i = 0; i < kWindow; ++i) {
+      const uint32_t v = wait_ready(col + int64_t(max(p - i, 0)) * stride, cur[i], ws);
+      excl += int(v & kValue);
+      if (v & kIncl) return excl;
+    }
+#pragma unroll
+    for (int i = 0; i < kWindow; ++i) cur[i] = nxt[i];
+  }
+  return excl;  // not reached: block 0 publishes an inclusive prefix
+}
+
+// kFromIdx: the picks are already in topk_idx (the router GEMM wrote them);
+// steps 2-5 run on them and topk_idx / topk_w are left as they are.
+template <int VPL, int VEC, bool kFromIdx>
+__global__ void __launch_bounds__(kLbThreads, 2) route_kernel(RouteArgs a) {
   __shared__ int32_t s_sel[kRouteTokens * kMaxTopK];  // picks of the block's tokens
   __shared__ uint32_t s_mask[kMaxExperts];            // token mask per expert
-  __shared__ int4 s_warp[kWarps];
-  __shared__ int32_t s_off[4];
-  __shared__ unsigned s_parity;
-  const int E = a.E, K = a.K;
+  __shared__ int32_t s_excl[kMaxExperts];             // exclusive prefix per expert
+  __shared__ int32_t s_wsum[kLbWarps];
+  __shared__ unsigned s_b, s_half, s_dirty;
+  const int E = a.E, K = a.K, B = a.blocks;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  Ctrl* ctrl = reinterpret_cast<Ctrl*>(a.ws);
   grid_dependency_wait();
-  // This call's half of the totals: the barrier generation's parity, read
-  // before any block can reach the barrier that bumps it.
-  if (tid == 0) s_parity = ld_acquire_gpu(&reinterpret_cast<Ctrl*>(a.ws)->gen) & 1u;
+  if (tid == 0) {
+    // the half and the rows to clear are read before the ticket is taken;
+    // the last block changes them only after every ticket is out
+    const unsigned half = a.flag_halves == 2 ? (ld_acquire_gpu(&ctrl->parity) & 1u) : 0u;
+    s_half = half;
+    s_dirty = a.flag_halves == 2 ? ld_relaxed_gpu(&ctrl->dirty[half ^ 1u]) : 0u;
+    s_b = atomicAdd(&ctrl->ticket, 1u);
+  }
+  for (int e = tid; e < E; e += kLbThreads) s_mask[e] = 0u;
   __syncthreads();
-  int32_t* tot = a.totals + size_t(s_parity) * E;
-
-  // ---- phase 1: route blocks b = blockIdx.x, blockIdx.x + grid, ...
-  for (int b = blockIdx.x; b < a.blocks; b += gridDim.x) {
-    const int t_base = b * kRouteTokens;
-    const int valid = max(0, min(kRouteTokens, a.n - t_base));
-    for (int i = tid; i < E; i += kRouteThreads) s_mask[i] = 0;
-    if (warp < valid) {
-      const int e = route_token<VPL, VEC>(a, int64_t(t_base) + warp, lane);
-      if (lane < K) s_sel[warp * K + lane] = e;
-    }
-    __syncthreads();
-    for (int p = tid; p < valid * K; p += kRouteThreads)
-      atomicOr(&s_mask[s_sel[p]], 1u << (p / K));
-    __syncthreads();
-    for (int p = tid; p < valid * K; p += kRouteThreads) {
-      const int tl = p / K;
-      a.rank[int64_t(t_base) * K + p] = uint8_t(__popc(s_mask[s_sel[p]] & ((1u << tl) - 1u)));
-    }
-    for (int e = tid; e < E; e += kRouteThreads) {
-      const int c = __popc(s_mask[e]);
-      a.blk[int64_t(b) * E + e] = c;
-      if (c) atomicAdd(tot + e, c);  // integer sums: the order does not matter
-    }
-    __syncthreads();
+  const int b = int(s_b);
+  if (b >= B) {  // the counter was not reset: the workspace needs moe_workspace_init
+    if (tid == 0) set_status(a.ws, MOE_ERR_TIMEOUT);
+    return;
   }
+  uint32_t* flags = a.flags + size_t(s_half) * a.flag_rows * E;
+  const int t0 = b * kRouteTokens;
+  const int valid = max(0, min(kRouteTokens, a.n - t0));
 
-  if (!grid_barrier(a.ws, gridDim.x)) return;
-
-  // ---- phase 2: column units u = blockIdx.x, blockIdx.x + grid, ...
-  if ((E & 3) == 0) {
-    for (int u = blockIdx.x; u < E / 4; u += gridDim.x) scan_column<4>(a, u, tot, s_warp, s_off);
+  // ---- 1. top-k and softmax: warp w routes tokens w, w + kLbWarps, ...
+  if constexpr (kFromIdx) {
+    for (int p = tid; p < valid * K; p += kLbThreads) {
+      int e = __ldg(a.topk_idx + int64_t(t0) * K + p);
+      if (e < 0 || e >= E) {
+        set_status(a.ws, MOE_ERR_DEVICE_INDEX);
+        e = -1;
+      }
+      s_sel[p] = e;
+    }
   } else {
-    for (int u = blockIdx.x; u < E; u += gridDim.x) scan_column<1>(a, u, tot, s_warp, s_off);
-  }
-  if (blockIdx.x == 0) {
-    // the other halves start the next call (of either route kernel) at zero
-    int32_t* next = a.totals + size_t(s_parity ^ 1u) * E;
-    for (int e = tid; e < E; e += kRouteThreads) next[e] = 0;
-    if (a.masks) {
-      uint32_t* m = a.masks + size_t(s_parity ^ 1u) * a.mask_rows * E;
-      for (int i = tid; i < a.mask_rows * E; i += kRouteThreads) m[i] = 0u;
+    uint32_t key[kTokPerWarp][VPL];
+#pragma unroll
+    for (int i = 0; i < kTokPerWarp; ++i) {
+      const int tl = warp + i * kLbWarps;
+      if (tl < valid) load_keys<VPL, VEC, true>(a.logits + int64_t(t0 + tl) * E, E, lane, key[i]);
     }
-    if (tid == 0) a.expert_off[E] = a.R * a.region_rows;
+#pragma unroll
+    for (int i = 0; i < kTokPerWarp; ++i) {
+      const int tl = warp + i * kLbWarps;
+      if (tl < valid) {
+        float w;
+        bool nonfinite;
+        const int e = select_topk<VPL, VEC>(key[i], K, lane, &w, &nonfinite);
+        if (lane < K) {
+          const int64_t tk = int64_t(t0 + tl) * K + lane;
+          a.topk_idx[tk] = e;
+          a.topk_w[tk] = w;
+          s_sel[tl * K + lane] = e;
+        }
+        if (nonfinite && lane == 0) set_status(a.ws, MOE_ERR_NONFINITE);
+      }
+    }
+  }
+  __syncthreads();
+  // ---- 2. per-expert token masks of the block
+  for (int p = tid; p < valid * K; p += kLbThreads)
+    if (!kFromIdx || s_sel[p] >= 0) atomicOr(&s_mask[s_sel[p]], 1u << (p / K));
+  __syncthreads();
+  // ---- 3. publish, look back, publish the inclusive prefix
+  // (every column's aggregate goes out before any of this thread's waits)
+  for (int e = tid; e < E; e += kLbThreads)
+    st_relaxed_u32(flags + int64_t(b) * E + e,
+                   (b == 0 ? kReady | kIncl : kReady) | uint32_t(__popc(s_mask[e])));
+  for (int e = tid; e < E; e += kLbThreads) {
+    int excl = 0;
+    if (b > 0) {
+      excl = look_back(flags + e, b, E, a.ws);
+      st_relaxed_u32(flags + int64_t(b) * E + e,
+                     kReady | kIncl | uint32_t(excl + __popc(s_mask[e])));
+    }
+    s_excl[e] = excl;
+  }
+  // the rows of the other half that the previous call wrote start the next
+  // call at zero; route blocks share them out
+  if (a.flag_halves == 2) {
+    uint32_t* other = a.flags + size_t(s_half ^ 1u) * a.flag_rows * E;
+    for (int r = b; r < int(s_dirty); r += B)
+      for (int e = tid; e < E; e += kLbThreads) other[int64_t(r) * E + e] = 0u;
+  }
+  __syncthreads();
+  // ---- 4. in-expert positions of the block's picks
+  for (int p = tid; p < valid * K; p += kLbThreads) {
+    const int e = s_sel[p];
+    a.pos[int64_t(t0) * K + p] =
+        kFromIdx && e < 0 ? -1 : s_excl[e] + __popc(s_mask[e] & ((1u << (p / K)) - 1u));
+  }
+  // ---- 5. the last block: totals -> rank-major offsets
+  if (b == B - 1) {
+    // exclusive scan of the totals over the experts (kExpPerThread per thread)
+    int tot[kExpPerThread];
+    int sum = 0;
+#pragma unroll
+    for (int i = 0; i < kExpPerThread; ++i) {
+      const int e = tid * kExpPerThread + i;
+      tot[i] = e < E ? s_excl[e] + __popc(s_mask[e]) : 0;
+      sum += tot[i];
+    }
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(kFull, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) s_wsum[warp] = incl;
+    __syncthreads();
+    int before = 0;
+    for (int w2 = 0; w2 < warp; ++w2) before += s_wsum[w2];
+    int pre = before + incl - sum;  // totals of the experts below this thread's first
+    __syncthreads();                // s_excl is rewritten below
+#pragma unroll
+    for (int i = 0; i < kExpPerThread; ++i) {
+      const int e = tid * kExpPerThread + i;
+      if (e < E) s_excl[e] = pre;  // now: prefix of totals over all experts below e
+      pre += tot[i];
+    }
+    __syncthreads();
+    const int per_rank = E / a.R;
+#pragma unroll
+    for (int i = 0; i < kExpPerThread; ++i) {
+      const int e = tid * kExpPerThread + i;
+      if (e < E) {
+        const int r = e / per_rank;
+        const int off = r * a.region_rows + s_excl[e] - s_excl[r * per_rank];
+        a.counts[e] = tot[i];
+        a.expert_off[e] = off;
+        a.off[e] = off;
+      }
+    }
+    if (tid == 0) {
+      a.expert_off[E] = a.R * a.region_rows;
+      a.off[E] = a.R * a.region_rows;
+      if (a.flag_halves == 2) {
+        ctrl->dirty[s_half] = unsigned(B);
+        ctrl->parity = s_half ^ 1u;
+      }
+      ctrl->ticket = 0u;
+    }
   }
   grid_dependents_launch();
 }
 
-// Cooperative launch: every block resident, as the grid barrier requires.
-template <int VPL, int VEC>
-cudaError_t launch_coop(const RouteArgs& a, int sms, cudaStream_t st) {
-  static std::atomic<int> per_sm[64];  // resident blocks per SM, per device (0 = unknown)
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev >= 64) return cudaErrorInvalidDevice;
-  int nb_known = per_sm[dev].load(std::memory_order_relaxed);
-  if (nb_known == 0) {
-    int nb = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, route_kernel<VPL, VEC>, kRouteThreads, 0);
-    if (e != cudaSuccess) return e;
-    if (nb < 1) return cudaErrorInvalidConfiguration;
-    per_sm[dev].store(nb, std::memory_order_relaxed);
-    nb_known = nb;
-  }
-  const int cols = (a.E & 3) == 0 ? a.E / 4 : a.E;
-  int grid = a.blocks > cols ? a.blocks : cols;
-  if (grid > nb_known * sms) grid = nb_known * sms;
-  return launch_cooperative(route_kernel<VPL, VEC>, dim3(unsigned(grid)), dim3(kRouteThreads), 0,
-                            st, a);
+template <int VPL, int VEC, bool kFromIdx>
+cudaError_t launch_lb(const RouteArgs& a, cudaStream_t st) {
+  return launch_pdl(route_kernel<VPL, VEC, kFromIdx>, dim3(unsigned(a.blocks)), dim3(kLbThreads), 0,
+                    st, a);
+}
+
+cudaError_t launch_with(RouteArgs& a, const moe_plan& p, int32_t n, cudaStream_t st,
+                        bool from_idx = false) {
+  a.n = n;
+  a.E = p.d.n_experts;
+  a.K = p.d.top_k;
+  a.R = p.d.n_ranks;
+  a.blocks = route_blocks(n);
+  a.region_rows = int32_t(region_rows(p, n));
+  a.masks = nullptr;
+  a.mask_rows = 0;
+  if (from_idx) return launch_lb<1, 1, true>(a, st);
+  return with_route_shape(a.E, [&](auto vpl, auto vec) {
+    return launch_lb<decltype(vpl)::value, decltype(vec)::value, false>(a, st);
+  });
 }
 
 }  // namespace
@@ -233,59 +295,51 @@ cudaError_t launch_route(const moe_plan& p, int32_t n, const float* logits, int3
   a.topk_w = topk_w;
   a.counts = counts;
   a.expert_off = expert_off;
-  a.blk = reinterpret_cast<int32_t*>(w + p.lay.blk);
-  a.bases = reinterpret_cast<int32_t*>(w + p.lay.bases);
-  a.totals = reinterpret_cast<int32_t*>(w + p.lay.totals);
-  a.masks = reinterpret_cast<uint32_t*>(w + p.lay.masks);
-  a.mask_rows = mask_rows(p);
-  a.rank = reinterpret_cast<uint8_t*>(w + p.lay.rank);
+  a.flags = reinterpret_cast<uint32_t*>(w + p.lay.flags);
+  a.flag_halves = 2;
+  a.flag_rows = p.blocks_max;
+  a.pos = reinterpret_cast<int32_t*>(w + p.lay.pos);
+  a.off = reinterpret_cast<int32_t*>(w + p.lay.off);
   a.ws = ws;
-  a.n = n;
-  a.E = p.d.n_experts;
-  a.K = p.d.top_k;
-  a.R = p.d.n_ranks;
-  a.blocks = route_blocks(n);
-  a.region_rows = int32_t(region_rows(p, n));
-  const int sms = num_sms();
-  return with_route_shape(a.E, [&](auto vpl, auto vec) {
-    return launch_coop<decltype(vpl)::value, decltype(vec)::value>(a, sms, st);
-  });
+  return launch_with(a, p, n, st);
 }
 
-}  // namespace moe
+// Counts, offsets and positions of picks already in topk_idx (the workspace
+// path of launch_route without its top-k step).
+cudaError_t launch_route_counts(const moe_plan& p, int32_t n, int32_t* topk_idx, int32_t* counts,
+                                int32_t* expert_off, void* ws, cudaStream_t st) {
+  char* w = static_cast<char*>(ws);
+  RouteArgs a;
+  a.logits = nullptr;
+  a.topk_idx = topk_idx;
+  a.topk_w = nullptr;
+  a.counts = counts;
+  a.expert_off = expert_off;
+  a.flags = reinterpret_cast<uint32_t*>(w + p.lay.flags);
+  a.flag_halves = 2;
+  a.flag_rows = p.blocks_max;
+  a.pos = reinterpret_cast<int32_t*>(w + p.lay.pos);
+  a.off = reinterpret_cast<int32_t*>(w + p.lay.off);
+  a.ws = ws;
+  return launch_with(a, p, n, st, true);
+}
 
-namespace moe {
-
-// The route kernels on caller-chosen scratch: ctrl (control words), blk and
-// bases ([route blocks, E] int32 each), totals ([2, E] int32, zero before the
-// first call) and rank ([n, k] bytes).
 cudaError_t launch_route_on(const moe_plan& p, int32_t n, const float* logits, int32_t* topk_idx,
                             float* topk_w, int32_t* counts, int32_t* expert_off, void* ctrl,
-                            int32_t* blk, int32_t* bases, int32_t* totals, uint32_t* masks,
-                            uint8_t* rank, cudaStream_t st) {
+                            uint32_t* flags, int32_t* pos, int32_t* off, cudaStream_t st) {
   RouteArgs a;
   a.logits = logits;
   a.topk_idx = topk_idx;
   a.topk_w = topk_w;
   a.counts = counts;
   a.expert_off = expert_off;
-  a.blk = blk;
-  a.bases = bases;
-  a.totals = totals;
-  a.masks = masks;
-  a.mask_rows = mask_rows(p);
-  a.rank = rank;
+  a.flags = flags;
+  a.flag_halves = 1;
+  a.flag_rows = route_blocks(n);
+  a.pos = pos;
+  a.off = off;
   a.ws = ctrl;
-  a.n = n;
-  a.E = p.d.n_experts;
-  a.K = p.d.top_k;
-  a.R = p.d.n_ranks;
-  a.blocks = route_blocks(n);
-  a.region_rows = int32_t(region_rows(p, n));
-  const int sms = num_sms();
-  return with_route_shape(a.E, [&](auto vpl, auto vec) {
-    return launch_coop<decltype(vpl)::value, decltype(vec)::value>(a, sms, st);
-  });
+  return launch_with(a, p, n, st);
 }
 
 }  // namespace moe

@@ -19,12 +19,16 @@ struct RouteArgs {
   float* topk_w;
   int32_t* counts;
   int32_t* expert_off;
-  int32_t* blk;    // [blocks, E] per-block counts
-  int32_t* bases;  // [blocks, E] per-block absolute base slots
-  int32_t* totals; // [2, E] expert totals, the half of this call chosen by barrier parity
+  // route kernel: [halves, rows, E] look-back words (one half per call when
+  // halves == 2, alternating, the other half cleared for the next call), the
+  // in-expert position of every pick [n, k] and a copy of the offsets [E + 1]
+  uint32_t* flags;
+  int32_t flag_halves;  // 2 (workspace: alternate halves) or 1 (pre-zeroed, noalloc)
+  int32_t flag_rows;    // rows per half
+  int32_t* pos;
+  int32_t* off;
   uint32_t* masks; // [2, mask_rows, E] token masks of the fused kernel (null: none)
   int32_t mask_rows;
-  uint8_t* rank;   // [n, k]: rank of (t, j) among the block's tokens picking e
   void* ws;
   int32_t n, E, K, R;
   int32_t blocks;       // route blocks B = ceil(n / 32), at least 1
@@ -56,14 +60,12 @@ __device__ __forceinline__ int expert_of(int q, int lane) {
   else return q * 32 + lane;
 }
 
-// Top-k and softmax of one logit row by the calling warp: lane j < K gets
-// pick j and its weight; *nonfinite tells whether a pick had a non-finite
-// logit (fewer than K finite values in the row).  kStream loads the row as
-// read-once data; otherwise it stays cached for other blocks reading it too.
+// The logits of one row as order-preserving keys, in the lane layout of
+// expert_of.  kStream loads the row as read-once data; otherwise it stays
+// cached for other blocks reading it too.
 template <int VPL, int VEC, bool kStream>
-__device__ __forceinline__ int route_row(const float* row, int E, int K, int lane, float* w,
-                                         bool* nonfinite) {
-  uint32_t key[VPL];
+__device__ __forceinline__ void load_keys(const float* row, int E, int lane,
+                                          uint32_t (&key)[VPL]) {
   if constexpr (VEC == 4) {
 #pragma unroll
     for (int q4 = 0; q4 < VPL / 4; ++q4) {
@@ -81,6 +83,14 @@ __device__ __forceinline__ int route_row(const float* row, int E, int K, int lan
       key[q] = e < E ? order_key(kStream ? __ldcs(row + e) : __ldg(row + e)) : 0u;
     }
   }
+}
+
+// Top-k and softmax of one row's keys by the calling warp: lane j < K gets
+// pick j and its weight; *nonfinite tells whether a pick had a non-finite
+// logit (fewer than K finite values in the row).
+template <int VPL, int VEC>
+__device__ __forceinline__ int select_topk(const uint32_t (&key)[VPL], int K, int lane, float* w,
+                                           bool* nonfinite) {
   // This lane's best two untaken values (strict compares keep the lower id
   // first among equal keys).  Each round the warp takes the largest head;
   // the owning lane moves its second value up, and rescans only when both
@@ -138,19 +148,14 @@ __device__ __forceinline__ int route_row(const float* row, int E, int K, int lan
   return my_i;
 }
 
-// Top-k and softmax of token t by the calling warp, written to topk_idx and
-// topk_w; returns lane j's pick.
-template <int VPL, int VEC>
-__device__ __forceinline__ int route_token(const RouteArgs& a, int64_t t, int lane) {
-  float w;
-  bool nonfinite;
-  const int e = route_row<VPL, VEC, true>(a.logits + t * a.E, a.E, a.K, lane, &w, &nonfinite);
-  if (lane < a.K) {
-    a.topk_idx[t * a.K + lane] = e;
-    a.topk_w[t * a.K + lane] = w;
-  }
-  if (nonfinite && lane == 0) set_status(a.ws, MOE_ERR_NONFINITE);
-  return e;
+// Top-k and softmax of one logit row by the calling warp (load_keys, then
+// select_topk).
+template <int VPL, int VEC, bool kStream>
+__device__ __forceinline__ int route_row(const float* row, int E, int K, int lane, float* w,
+                                         bool* nonfinite) {
+  uint32_t key[VPL];
+  load_keys<VPL, VEC, kStream>(row, E, lane, key);
+  return select_topk<VPL, VEC>(key, K, lane, w, nonfinite);
 }
 
 // Calls f(VPL, VEC) -- as std::integral_constant values -- with the logits

@@ -7,9 +7,10 @@
 
 namespace {
 
-// Scratch of moe_route_topk_noalloc: the control words, the per-block count
-// and base tables and the per-token ranks of one call.  Every GPU that loads
-// this library holds these bytes until the process exits.
+// Scratch of moe_route_topk_noalloc: the control words, the look-back words
+// of the route blocks, the in-expert positions of the picks and a copy of the
+// offsets of one call.  Every GPU that loads this library holds these bytes
+// until the process exits.
 static __device__ __align__(256) unsigned char g_route_scratch[MOE_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
@@ -38,11 +39,27 @@ cudaError_t scratch_address(void** out) {
 
 }  // namespace
 
+namespace {
+
+// Byte offsets inside the scratch array for a call with n tokens.
+struct NoallocLayout {
+  size_t flags, pos, off, end;
+};
+
+NoallocLayout noalloc_layout(const moe_plan& p, int32_t n) {
+  NoallocLayout L;
+  L.flags = sizeof(moe::Ctrl);
+  L.pos = L.flags + moe::align256(size_t(moe::route_blocks(n)) * p.d.n_experts * 4);
+  L.off = L.pos + moe::align256(size_t(n) * p.d.top_k * 4);
+  L.end = L.off + moe::align256(size_t(p.d.n_experts + 1) * 4);
+  return L;
+}
+
+}  // namespace
+
 extern "C" MOE_API size_t moe_route_topk_noalloc_bytes(const moe_plan* p, int32_t n) {
   if (!p || n < 0) return 0;
-  const size_t table = moe::align256(size_t(moe::route_blocks(n)) * p->d.n_experts * 4);
-  const size_t totals = moe::align256(size_t(2) * p->d.n_experts * 4);
-  return sizeof(moe::Ctrl) + totals + 2 * table + moe::align256(size_t(n) * p->d.top_k);
+  return noalloc_layout(*p, n).end;
 }
 
 extern "C" MOE_API moe_status moe_route_topk_noalloc(const moe_plan* p, int32_t n,
@@ -53,23 +70,32 @@ extern "C" MOE_API moe_status moe_route_topk_noalloc(const moe_plan* p, int32_t 
   if (!counts || !expert_off || (n > 0 && (!logits || !topk_idx || !topk_w)))
     return MOE_ERR_INVALID_ARG;
   if (n > 0 && (reinterpret_cast<uintptr_t>(logits) & 15u)) return MOE_ERR_INVALID_ARG;
-  if (moe_route_topk_noalloc_bytes(p, n) > MOE_NOALLOC_SCRATCH_BYTES) return MOE_ERR_WORKSPACE;
+  const NoallocLayout L = noalloc_layout(*p, n);
+  if (L.end > MOE_NOALLOC_SCRATCH_BYTES) return MOE_ERR_WORKSPACE;
   void* base = nullptr;
   if (scratch_address(&base) != cudaSuccess) return MOE_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   char* b = static_cast<char*>(base);
-  const size_t table = moe::align256(size_t(moe::route_blocks(n)) * p->d.n_experts * 4);
-  const size_t totals_bytes = moe::align256(size_t(2) * p->d.n_experts * 4);
-  int32_t* totals = reinterpret_cast<int32_t*>(b + sizeof(moe::Ctrl));
-  int32_t* blk = reinterpret_cast<int32_t*>(b + sizeof(moe::Ctrl) + totals_bytes);
-  int32_t* bases = reinterpret_cast<int32_t*>(b + sizeof(moe::Ctrl) + totals_bytes + table);
-  uint8_t* rank = reinterpret_cast<uint8_t*>(b + sizeof(moe::Ctrl) + totals_bytes + 2 * table);
-  // The array keeps whatever the previous call left; the control words and
-  // the expert totals must start at zero.  The tables are fully rewritten.
-  if (cudaMemsetAsync(b, 0, sizeof(moe::Ctrl) + totals_bytes, st) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  const cudaError_t e = moe::launch_route_on(*p, n, logits, topk_idx, topk_w, counts, expert_off,
-                                             b, blk, bases, totals, nullptr, rank, st);
+  // The array keeps whatever the previous call left: the control words
+  // (status, ticket) and this call's look-back words must start at zero.
+  // The positions and offsets are fully rewritten.
+  if (cudaMemsetAsync(b, 0, L.pos, st) != cudaSuccess) return MOE_ERR_CUDA;
+  const cudaError_t e = moe::launch_route_on(
+      *p, n, logits, topk_idx, topk_w, counts, expert_off, b,
+      reinterpret_cast<uint32_t*>(b + L.flags), reinterpret_cast<int32_t*>(b + L.pos),
+      reinterpret_cast<int32_t*>(b + L.off), st);
   if (e == cudaSuccess) return MOE_OK;
   return e == cudaErrorNotSupported ? MOE_ERR_UNSUPPORTED : MOE_ERR_CUDA;
+}
+
+extern "C" MOE_API moe_status moe_route_topk_noalloc_status(moe_stream_t stream) {
+  void* base = nullptr;
+  if (scratch_address(&base) != cudaSuccess) return MOE_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int v = 0;
+  if (cudaMemcpyAsync(&v, &static_cast<moe::Ctrl*>(base)->status, sizeof(int),
+                      cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+  return static_cast<moe_status>(v);
 }

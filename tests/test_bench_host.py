@@ -104,3 +104,63 @@ def test_clock_sampler_window_and_short_region_fallback():
     s.proc = _Proc()
     rec = s.stop(1.031, 1.032)  # between samples: the two nearest
     assert rec["samples"] == 2 and rec["window"].startswith("nearest")
+
+
+def test_percentiles_nearest_rank():
+    sys.path.insert(0, ROOT)
+    import bench
+    p = bench.percentiles([5.0, 1.0, 4.0, 2.0, 3.0, 10.0, 6.0, 7.0, 8.0, 9.0, 0.0])
+    assert (p["n"], p["min"], p["max"], p["p50"]) == (11, 0.0, 10.0, 5.0)
+    assert (p["p10"], p["p90"]) == (1.0, 9.0)
+    assert bench.percentiles([]) == {}
+
+
+def test_path_dtype_names_what_the_path_moves():
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads
+    d = bench.path_dtype(workloads.CONFIGS["prefill"])
+    assert d.startswith("fp8_e4m3 + fp32 scale per 128 cols rows") and "fp32 accumulate" in d
+    assert "bf16 Y / bf16 out" in d
+    assert bench.path_dtype(workloads.CONFIGS["tiny"]).startswith("fp32 rows")
+
+
+def test_oracle_on_host_cores_splits_the_batch():
+    """OracleCores runs the unchanged oracle in worker processes, one slice
+    of the batch each: two workers on the tiny workload start, answer every
+    step with a positive wall time, and cover all tokens; host_cpu names the
+    cores and the CPU model the numbers come from."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads
+    import oracle
+    oracle.build()
+    cfg = workloads.CONFIGS["tiny"]
+    pool = bench.OracleCores(cfg, bench.oracle_inputs(cfg, 64), workers=2)
+    try:
+        assert pool.workers == 2 and pool.tokens == 64
+        walls = [pool.step() for _ in range(2)]
+    finally:
+        pool.close()
+    assert all(w > 0 for w in walls)
+    host = bench.host_cpu()
+    assert host["cores_available"] >= 1 and host["nproc"] >= 1
+    assert "cpu_model" in host
+
+
+def test_reference_line_reports_measured_steps(capsys):
+    """The reference arm's ms_per_step is the measured time of the steps it
+    ran on its sample (tokens_per_step), so steps x ms_per_step is time that
+    was spent; value = sampled tokens / step time."""
+    sys.path.insert(0, ROOT)
+    import json
+    import bench
+    import oracle
+    oracle.build()
+    bench.main(["--impl", "reference", "--workload", "tiny", "--steps", "3", "--warmup", "3"])
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["steps"] == 3
+    assert line["tokens_per_step"] <= 64
+    assert line["value"] == pytest.approx(line["tokens_per_step"] / (line["ms_per_step"] * 1e-3))
+    assert line["cpu_baseline"]["cores"] >= 1 and "cpu_model" in line["cpu_baseline"]
+    assert line["step_ms"]["n"] == 3

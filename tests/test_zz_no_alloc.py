@@ -20,6 +20,7 @@ import workloads
 pytestmark = pytest.mark.gpu
 
 MOE_ERR_WORKSPACE = -4
+MOE_ERR_NONFINITE = -7
 
 
 def _lib():
@@ -30,6 +31,8 @@ def _lib():
     lib.moe_route_topk_noalloc.argtypes = [P, i32, P, P, P, P, P, P]
     lib.moe_route_topk_noalloc_bytes.restype = ctypes.c_size_t
     lib.moe_route_topk_noalloc_bytes.argtypes = [P, i32]
+    lib.moe_route_topk_noalloc_status.restype = ctypes.c_int
+    lib.moe_route_topk_noalloc_status.argtypes = [P]
     return mr, lib
 
 
@@ -87,3 +90,56 @@ def test_noalloc_refuses_calls_beyond_its_scratch():
     assert rc == MOE_ERR_WORKSPACE
     torch.cuda.synchronize()
     assert bool((out["counts"] == -9).all())  # nothing ran
+
+
+def test_noalloc_zero_tokens_then_a_batch():
+    """n = 0 returns MOE_OK with zero counts and offsets (as moe_route_topk
+    does), and a following call with tokens still matches the workspace call."""
+    mr, lib = _lib()
+    cfg = workloads.CONFIGS["decode"]
+    n = 128
+    dev = torch.device("cuda", 0)
+    plan = mr.Plan.from_config(cfg, n_max=n)
+    stream = torch.cuda.current_stream(dev)
+    ws = plan.new_workspace(dev)
+    empty = torch.empty(0, cfg.n_experts, device=dev)
+    ref0, got0 = plan.new_buffers(1, dev), plan.new_buffers(1, dev)
+    got0["counts"].fill_(-1)
+    got0["expert_off"].fill_(-1)
+    mr.moe_route_topk(plan, empty, ref0["topk_idx"][:0], ref0["topk_w"][:0], ref0["counts"],
+                      ref0["expert_off"], ws)
+    assert _route_noalloc(lib, plan, empty, got0, stream) == 0
+    torch.cuda.synchronize()
+    assert lib.moe_route_topk_noalloc_status(ctypes.c_void_p(stream.cuda_stream)) == 0
+    assert bool((got0["counts"] == 0).all())
+    assert torch.equal(got0["expert_off"], ref0["expert_off"])
+    logits = workloads.make_inputs(cfg, seed=23, n=n)["logits"].to(dev)
+    ref, got = plan.new_buffers(n, dev), plan.new_buffers(n, dev)
+    mr.moe_route_topk(plan, logits, ref["topk_idx"], ref["topk_w"], ref["counts"],
+                      ref["expert_off"], ws)
+    assert _route_noalloc(lib, plan, logits, got, stream) == 0
+    torch.cuda.synchronize()
+    for key in ("topk_idx", "counts", "expert_off"):
+        assert torch.equal(got[key], ref[key]), key
+    assert mr.moe_get_status(plan, ws) == 0
+
+
+def test_noalloc_status_reports_the_last_call():
+    """A logit row with fewer than k finite values is a device-detected error
+    of the allocation-free call too: moe_route_topk_noalloc_status reports it,
+    and the next clean call starts again from MOE_OK."""
+    mr, lib = _lib()
+    cfg = workloads.CONFIGS["tiny"]
+    n = 64
+    dev = torch.device("cuda", 0)
+    plan = mr.Plan.from_config(cfg, n_max=n)
+    stream = torch.cuda.current_stream(dev)
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    logits = workloads.make_inputs(cfg, seed=24, n=n)["logits"]
+    bad = logits.clone()
+    bad[5, :] = float("nan")
+    out = plan.new_buffers(n, dev)
+    assert _route_noalloc(lib, plan, bad.to(dev), out, stream) == 0
+    assert lib.moe_route_topk_noalloc_status(sp) == MOE_ERR_NONFINITE
+    assert _route_noalloc(lib, plan, logits.to(dev), out, stream) == 0
+    assert lib.moe_route_topk_noalloc_status(sp) == 0
