@@ -64,14 +64,13 @@ Layout make_layout(const moe_plan& p) {
     return here;
   };
   L.ctrl = take(sizeof(Ctrl));
-  // right after ctrl, all cleared together by moe_workspace_init: the route
-  // kernel's look-back words [2, route blocks, E] (alternate halves per call)
-  // and the fused kernel's token masks [2, mask rows, E] (alternate halves by
-  // its grid-barrier generation)
-  L.flags = take(size_t(2) * p.blocks_max * d.n_experts * 4);
+  // right after ctrl, cleared with it by moe_workspace_init: the fused
+  // kernel's token masks [2, mask rows, E] (alternate halves by its
+  // grid-barrier generation)
   L.masks = take(size_t(2) * mask_rows(p) * d.n_experts * 4);
-  L.pos = take(size_t(d.n_max) * d.top_k * 4);
-  L.off = take(size_t(d.n_experts + 1) * 4);
+  L.blk = take(size_t(p.blocks_max) * d.n_experts * 4);
+  L.bases = take(size_t(p.blocks_max) * d.n_experts * 4);
+  L.rank = take(size_t(d.n_max) * d.top_k);
   L.route_end = at;
   const size_t nk = size_t(d.n_max) * d.top_k;
   const size_t T = size_t(p.total_max);
@@ -117,8 +116,6 @@ moe_status moe_plan_create(const moe_desc* desc, moe_plan** out) {
   const moe_desc d = *desc;
   if (d.n_max < 1 || d.hidden < 1 || d.n_experts < 1 || d.top_k < 1 || d.n_ranks < 1)
     return MOE_ERR_INVALID_ARG;
-  // per-expert counts travel in 30-bit fields of the route kernel's look-back words
-  if (d.n_max >= (1 << 30)) return MOE_ERR_UNSUPPORTED;
   if (d.n_experts > kMaxExperts || d.top_k > kMaxTopK) return MOE_ERR_UNSUPPORTED;
   if (d.top_k > d.n_experts || d.n_experts % d.n_ranks != 0) return MOE_ERR_INVALID_ARG;
   auto dtype_ok = [](int t) { return t == MOE_F32 || t == MOE_BF16 || t == MOE_FP8_E4M3; };
@@ -412,8 +409,8 @@ moe_status moe_get_status(const moe_plan* p, void* ws, moe_stream_t stream) {
 
 moe_status moe_workspace_init(const moe_plan* p, void* ws, moe_stream_t stream) {
   if (!p || !ws) return MOE_ERR_INVALID_ARG;
-  // control words, look-back words and token masks (which follow them)
-  return cudaMemsetAsync(ws, 0, p->lay.pos, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+  // control words and token masks (which follow them)
+  return cudaMemsetAsync(ws, 0, p->lay.blk, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
              ? MOE_OK
              : MOE_ERR_CUDA;
 }

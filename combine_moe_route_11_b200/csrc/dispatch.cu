@@ -9,9 +9,8 @@
 // divides both the 7168-byte FP8 rows and the 14336-byte bf16 rows of the
 // workloads, and 32 registers per thread let 8 blocks share an SM.  Every
 // lane loads 2 sixteen-byte vectors of the chunk first (they do not depend on
-// routing), while lanes j < k resolve the slot of choice j -- the expert's
-// offset plus the pick's in-expert position, both left in the workspace by
-// the route call, no metadata round trip --
+// routing), while lanes j < k resolve the slot of choice j -- the route
+// call's per-block base plus the in-block rank, no metadata round trip --
 // then the warp stores the chunk k times.  Scales and the index maps go with
 // the first chunk of the row.  High occupancy keeps enough loads and stores
 // in flight: on B200 this beats staging the chunks through shared memory
@@ -31,8 +30,8 @@ struct DispatchArgs {
   const uint8_t* x;
   const float* x_scale;
   const int32_t* topk_idx;
-  const int32_t* off;    // [E + 1] expert offsets (the route call's copy)
-  const int32_t* pos;    // [n, k] position of each pick inside its expert's segment
+  const int32_t* bases;  // [route blocks, E] absolute base slot of each block's run of an expert
+  const uint8_t* rank;   // [n, k] rank of each pick among its block's tokens picking the expert
   uint8_t* recv;
   float* recv_scale;
   int32_t* slot_of;
@@ -66,7 +65,7 @@ __global__ void __launch_bounds__(kThreads, 8) dispatch_kernel(DispatchArgs a) {
       const int64_t tk = t * a.K + lane;
       const int e = __ldg(a.topk_idx + tk);
       if (e >= 0 && e < a.E) {
-        slot = __ldg(a.off + e) + __ldg(a.pos + tk);
+        slot = __ldg(a.bases + (t / kRouteTokens) * a.E + e) + a.rank[tk];
         if (slot < 0 || slot >= a.total) slot = -1;
       }
       if (slot < 0) set_status(a.ws, MOE_ERR_DEVICE_INDEX);
@@ -122,8 +121,8 @@ cudaError_t launch_dispatch(const moe_plan& p, int32_t n, const void* x, const f
   a.x = static_cast<const uint8_t*>(x);
   a.x_scale = x_scale;
   a.topk_idx = topk_idx;
-  a.off = reinterpret_cast<const int32_t*>(static_cast<const char*>(ws) + p.lay.off);
-  a.pos = reinterpret_cast<const int32_t*>(static_cast<const char*>(ws) + p.lay.pos);
+  a.bases = reinterpret_cast<const int32_t*>(static_cast<const char*>(ws) + p.lay.bases);
+  a.rank = reinterpret_cast<const uint8_t*>(static_cast<const char*>(ws) + p.lay.rank);
   a.recv = static_cast<uint8_t*>(recv);
   a.recv_scale = recv_scale;
   a.slot_of = slot_of;

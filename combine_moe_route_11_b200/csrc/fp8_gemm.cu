@@ -131,10 +131,27 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
-// 8 consecutive fp32 columns of this thread's TMEM lane.  The 128
-// accumulators of a promotion thread and the temporaries of one load must fit
-// in 168 registers: 320 threads put three warps on one of the SM's four
-// register-file partitions of 16 K registers, so no thread may have more.
+// 16 consecutive fp32 columns of this thread's TMEM lane.  Each load waits
+// for its round trip to tensor memory, so wider loads mean fewer waits per
+// k-block; but the 128 accumulators of a promotion thread and the
+// temporaries of one load must fit in 168 registers (320 threads put three
+// warps on one of the SM's four register-file partitions of 16 K registers,
+// so no thread may have more), and 32 temporaries do not.  GEMM2 fits 16;
+// GEMM1, whose SwiGLU epilogue needs a few more, loads 8 at a time.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
   uint32_t r[8];
   asm volatile(
@@ -145,6 +162,20 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
   for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Folds 32 partial-sum columns, scaled by sc, into acc[0..32).
+template <bool kSwiGLU>
+__device__ __forceinline__ void promote32(uint32_t taddr, float sc, float* acc) {
+  constexpr int W = kSwiGLU ? 8 : 16;
+#pragma unroll
+  for (int h = 0; h < 32 / W; ++h) {
+    float v[W];
+    if constexpr (W == 8) tmem_ld8(taddr + uint32_t(h * W), v);
+    else tmem_ld16(taddr + uint32_t(h * W), v);
+#pragma unroll
+    for (int i = 0; i < W; ++i) acc[h * W + i] = fmaf(v[i], sc, acc[h * W + i]);
+  }
 }
 
 // The per-k-block waits of this kernel run about 50 times as often as the
@@ -381,14 +412,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const float sc = (kSwiGLU && j >= 2) ? s1 : s0;
-#pragma unroll
-          for (int hj = 0; hj < 4; ++hj) {
-            float v[8];
-            tmem_ld8(taddr + uint32_t(chunk_col<kSwiGLU>(half, j) + hj * 8), v);
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              acc[j * 32 + hj * 8 + i] = fmaf(v[i], sc, acc[j * 32 + hj * 8 + i]);
-          }
+          promote32<kSwiGLU>(taddr + uint32_t(chunk_col<kSwiGLU>(half, j)), sc, acc + j * 32);
         }
         tc_fence_before();
         __syncwarp();

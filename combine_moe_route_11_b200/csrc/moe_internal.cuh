@@ -20,19 +20,14 @@ constexpr int kMaxTopK = 32;
 // Largest batch, in route blocks, that the fused route + dispatch launch
 // takes (n <= 1024 tokens); larger batches run the two kernels.
 constexpr int kFusedMaxBlocks = 32;
-// Up to this many tokens the one launch needs no grid barrier either: every
-// block routes all tokens itself (route_dispatch_small_kernel).
-constexpr int kSmallMaxTokens = 256;
 
 // Control words at the start of every workspace.
 struct Ctrl {
   unsigned int arrive;    // fused kernel's grid barrier: blocks arrived (reset by the last one)
   int status;             // first device-detected error, 0 = none
   unsigned int gen;       // fused kernel's grid barrier: generation, bumped when all arrived
-  unsigned int ticket;    // route kernel: next route block to hand out (reset by the last one)
-  unsigned int parity;    // route kernel: half of the look-back table the next call uses
-  unsigned int dirty[2];  // route kernel: rows of each half the last call using it wrote
-  unsigned int pad[57];
+  unsigned int ticket;    // route kernel: route blocks done (reset by the last one)
+  unsigned int pad[60];
 };
 static_assert(sizeof(Ctrl) == 256, "control block is 256 bytes");
 
@@ -44,7 +39,7 @@ inline int elem_bytes(int dtype) {
 
 // Byte offsets of every buffer inside a workspace, fixed by n_max.
 struct Layout {
-  size_t ctrl, flags, masks, pos, off, route_end;  // [ctrl, pos) is cleared by moe_workspace_init
+  size_t ctrl, masks, blk, bases, rank, route_end;  // [ctrl, blk) is cleared by moe_workspace_init
   size_t topk_idx, topk_w, counts, expert_off, slot_of, src_of, recv, recv_scale, y, h;
   size_t hq, h_scale;  // FP8 SwiGLU experts: H in e4m3 and its per-128-column scales
   size_t end;
@@ -81,12 +76,12 @@ cudaError_t set_smem_limit(const void* kernel, int bytes);
 cudaError_t launch_route(const moe_plan& p, int32_t n, const float* logits, int32_t* topk_idx,
                          float* topk_w, int32_t* counts, int32_t* expert_off, void* ws,
                          cudaStream_t st);
-// The route kernel on caller-chosen scratch: ctrl (control words), flags
-// (one [route blocks, E] half of look-back words, zero before the call), pos
-// ([n, k] int32) and off ([E + 1] int32).
+// The route kernel on caller-chosen scratch: ctrl (control words, the
+// counter at zero), blk and bases ([route blocks, E] int32 each) and rank
+// ([n, k] bytes).
 cudaError_t launch_route_on(const moe_plan& p, int32_t n, const float* logits, int32_t* topk_idx,
                             float* topk_w, int32_t* counts, int32_t* expert_off, void* ctrl,
-                            uint32_t* flags, int32_t* pos, int32_t* off, cudaStream_t st);
+                            int32_t* blk, int32_t* bases, uint8_t* rank, cudaStream_t st);
 cudaError_t launch_route_counts(const moe_plan& p, int32_t n, int32_t* topk_idx, int32_t* counts,
                                 int32_t* expert_off, void* ws, cudaStream_t st);
 cudaError_t launch_router(const moe_plan& p, int32_t n, const void* x, const void* w_router,

@@ -19,14 +19,9 @@ struct RouteArgs {
   float* topk_w;
   int32_t* counts;
   int32_t* expert_off;
-  // route kernel: [halves, rows, E] look-back words (one half per call when
-  // halves == 2, alternating, the other half cleared for the next call), the
-  // in-expert position of every pick [n, k] and a copy of the offsets [E + 1]
-  uint32_t* flags;
-  int32_t flag_halves;  // 2 (workspace: alternate halves) or 1 (pre-zeroed, noalloc)
-  int32_t flag_rows;    // rows per half
-  int32_t* pos;
-  int32_t* off;
+  int32_t* blk;    // [blocks, E] per-block counts
+  int32_t* bases;  // [blocks, E] per-block absolute base slots
+  uint8_t* rank;   // [n, k]: rank of (t, j) among the block's tokens picking e
   uint32_t* masks; // [2, mask_rows, E] token masks of the fused kernel (null: none)
   int32_t mask_rows;
   void* ws;

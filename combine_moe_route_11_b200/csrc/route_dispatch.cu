@@ -187,178 +187,6 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_dispatch_kernel(FusedA
   grid_dependents_launch();
 }
 
-// ---------------------------------------------------------------- small batches
-// Up to kSmallMaxTokens tokens, every block routes EVERY token itself (the
-// logits are a few hundred kilobytes that stay in L2), so each block has all
-// the picks, masks, totals, offsets and bases in its own shared memory and
-// scatters its own tokens without waiting for any other block: no grid
-// barrier and no cooperative launch, an ordinary launch that the next kernel
-// can follow programmatically.  The redundant routing costs each block
-// n / 32 top-k selections per warp, which at decode sizes is less than a
-// barrier round trip.  Only the owner of a token writes its topk_idx /
-// topk_w; all blocks compute the same picks from the same logits with the
-// same code, so their slot tables agree.
-template <int VPL, int VEC>
-__global__ void __launch_bounds__(kRouteThreads, 1) route_dispatch_small_kernel(FusedArgs f) {
-  extern __shared__ int32_t s_dyn[];  // picks [n, K], masks [blocks, E], bases [blocks, E]
-  __shared__ int32_t s_pre[kMaxExperts];
-  __shared__ int32_t s_wsum[kWarps];
-  const RouteArgs& a = f.r;
-  const int E = a.E, K = a.K, B = a.blocks, n = a.n;
-  const int G = gridDim.x;
-  int32_t* s_pick = s_dyn;
-  uint32_t* s_mask = reinterpret_cast<uint32_t*>(s_dyn + n * K);
-  int32_t* s_base = s_dyn + n * K + B * E;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t row_bytes = int64_t(f.vecs) << 4;
-  const int mine = int(blockIdx.x) < n ? (n - 1 - int(blockIdx.x)) / G + 1 : 0;
-  const int items = mine * f.chunks;  // (owned token i, chunk c) -> i * chunks + c
-  grid_dependency_wait();
-
-  // ---- the first chunk of x, in flight while routing runs
-  uint4 v0 = make_uint4(0u, 0u, 0u, 0u);
-  if (warp < items) {
-    const int64_t t = blockIdx.x + int64_t(warp / f.chunks) * G;
-    const int64_t g = int64_t(warp % f.chunks) * 32 + lane;
-    if (g < f.vecs) v0 = ld_nc_v4(f.x + t * row_bytes + (g << 4));
-  }
-  for (int i = tid; i < B * E; i += kRouteThreads) s_mask[i] = 0u;
-  __syncthreads();
-
-  // ---- phase 1: every token, one warp per token
-  for (int t = warp; t < n; t += kWarps) {
-    float w;
-    bool nonfinite;
-    const int e = route_row<VPL, VEC, false>(a.logits + int64_t(t) * E, E, K, lane, &w, &nonfinite);
-    const bool owner = t % G == int(blockIdx.x);
-    if (lane < K) {
-      s_pick[t * K + lane] = e;
-      atomicOr(&s_mask[(t / kRouteTokens) * E + e], 1u << (t % kRouteTokens));
-      if (owner) {
-        a.topk_idx[int64_t(t) * K + lane] = e;
-        a.topk_w[int64_t(t) * K + lane] = w;
-      }
-    }
-    if (nonfinite && owner && lane == 0) set_status(a.ws, MOE_ERR_NONFINITE);
-  }
-  __syncthreads();
-
-  // ---- phase 2: totals, offsets and the base table, from the local masks
-  int tot = 0;
-  if (tid < E)
-    for (int b = 0; b < B; ++b) tot += __popc(s_mask[b * E + tid]);
-  int incl = tot;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(kFull, incl, o);
-    if (lane >= o) incl += y;
-  }
-  if (lane == 31) s_wsum[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    const int w = s_wsum[lane];
-    int wi = w;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(kFull, wi, o);
-      if (lane >= o) wi += y;
-    }
-    s_wsum[lane] = wi - w;
-  }
-  __syncthreads();
-  const int pre = incl - tot + s_wsum[warp];  // sum of the totals of experts below tid
-  if (tid < E) s_pre[tid] = pre;
-  __syncthreads();
-  if (tid < E) {
-    const int per_rank = E / a.R;
-    const int r = tid / per_rank;
-    const int off = r * a.region_rows + pre - s_pre[r * per_rank];
-    int run = off;
-    for (int b = 0; b < B; ++b) {
-      s_base[b * E + tid] = run;
-      run += __popc(s_mask[b * E + tid]);
-    }
-    if (blockIdx.x == 0) {
-      a.counts[tid] = tot;
-      a.expert_off[tid] = off;
-    }
-  }
-  if (blockIdx.x == 0 && tid == 0) a.expert_off[E] = a.R * a.region_rows;
-  __syncthreads();
-
-  // ---- phase 3: the chunks of this block's tokens to their k slots
-  for (int it = warp; it < items; it += kWarps) {
-    const int i = it / f.chunks, c = it % f.chunks;
-    const int t = int(blockIdx.x) + i * G;
-    const int64_t g = int64_t(c) * 32 + lane;
-    uint4 v = v0;
-    if (it != warp && g < f.vecs) v = ld_nc_v4(f.x + int64_t(t) * row_bytes + (g << 4));
-    int slot = -1;
-    if (lane < K) {
-      const int e = s_pick[t * K + lane];
-      if (e >= 0 && e < E) {
-        const int b = t / kRouteTokens, tl = t % kRouteTokens;
-        slot = s_base[b * E + e] + __popc(s_mask[b * E + e] & ((1u << tl) - 1u));
-        if (slot < 0 || slot >= f.total) slot = -1;
-      }
-      if (slot < 0) set_status(a.ws, MOE_ERR_DEVICE_INDEX);
-      if (c == 0) {
-        const int64_t tk = int64_t(t) * K + lane;
-        f.slot_of[tk] = slot;
-        if (slot >= 0) f.src_of[slot] = int32_t(tk);
-      }
-    }
-    for (int j = 0; j < K; ++j) {
-      const int s = __shfl_sync(kFull, slot, j);
-      if (s < 0) continue;  // uniform across the warp
-      if (g < f.vecs) st_cs_v4(f.recv + int64_t(s) * row_bytes + (g << 4), v);
-    }
-    if (c == 0 && f.S > 0) {
-      for (int i0 = 0; i0 < f.S; i0 += 32) {
-        const int si = i0 + lane;
-        const float sv = si < f.S ? __ldcs(f.x_scale + int64_t(t) * f.S + si) : 0.f;
-        for (int j = 0; j < K; ++j) {
-          const int s = __shfl_sync(kFull, slot, j);
-          if (s >= 0 && si < f.S) __stcs(f.recv_scale + int64_t(s) * f.S + si, sv);
-        }
-      }
-    }
-  }
-  grid_dependents_launch();
-}
-
-size_t small_smem(int n, int K, int blocks, int E) {
-  return (size_t(n) * K + 2 * size_t(blocks) * E) * 4;
-}
-
-template <int VPL, int VEC>
-cudaError_t launch_small(FusedArgs f, int sms, cudaStream_t st) {
-  static std::atomic<int> per_sm[64];  // resident blocks per SM, per device (0 = unknown)
-  const int kMaxDyn = int(small_smem(kSmallMaxTokens, kMaxTopK, kSmallMaxTokens / kRouteTokens,
-                                     kMaxExperts));
-  auto kernel = route_dispatch_small_kernel<VPL, VEC>;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev >= 64) return cudaErrorInvalidDevice;
-  e = set_smem_limit(reinterpret_cast<const void*>(kernel), kMaxDyn);
-  if (e != cudaSuccess) return e;
-  int nb_known = per_sm[dev].load(std::memory_order_relaxed);
-  if (nb_known == 0) {
-    int nb = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kernel, kRouteThreads, kMaxDyn);
-    if (e != cudaSuccess) return e;
-    if (nb < 1) return cudaErrorInvalidConfiguration;
-    per_sm[dev].store(nb, std::memory_order_relaxed);
-    nb_known = nb;
-  }
-  // one block per token, up to one wave
-  int64_t grid = f.r.n > 1 ? f.r.n : 1;
-  if (grid > int64_t(nb_known) * sms) grid = int64_t(nb_known) * sms;
-  return launch_pdl(kernel, dim3(unsigned(grid)), dim3(kRouteThreads),
-                    small_smem(f.r.n, f.r.K, f.r.blocks, f.r.E), st, f);
-}
-
 // Dynamic shared memory of a launch: masks and bases [blocks, E] and the
 // owned tokens' picks [owned, K].
 size_t fused_smem(int blocks, int E, int owned, int K) {
@@ -412,11 +240,9 @@ cudaError_t launch_route_dispatch(const moe_plan& p, int32_t n, const float* log
   a.topk_w = topk_w;
   a.counts = counts;
   a.expert_off = expert_off;
-  a.flags = nullptr;
-  a.flag_halves = 0;
-  a.flag_rows = 0;
-  a.pos = nullptr;
-  a.off = nullptr;
+  a.blk = nullptr;
+  a.bases = nullptr;
+  a.rank = nullptr;
   a.masks = reinterpret_cast<uint32_t*>(w + p.lay.masks);
   a.mask_rows = mask_rows(p);
   a.ws = ws;
@@ -437,12 +263,8 @@ cudaError_t launch_route_dispatch(const moe_plan& p, int32_t n, const float* log
   f.chunks = (f.vecs + 31) / 32;
   f.total = int32_t(total_rows(p, n));
   f.owned = 0;
-  const int sms = num_sms();
-  if (n <= kSmallMaxTokens)
-    return with_route_shape(a.E, [&](auto vpl, auto vec) {
-      return launch_small<decltype(vpl)::value, decltype(vec)::value>(f, sms, st);
-    });
   if (a.blocks > a.mask_rows) return cudaErrorInvalidValue;
+  const int sms = num_sms();
   return with_route_shape(a.E, [&](auto vpl, auto vec) {
     return launch_fused<decltype(vpl)::value, decltype(vec)::value>(f, sms, st);
   });

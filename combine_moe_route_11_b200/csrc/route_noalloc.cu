@@ -7,10 +7,9 @@
 
 namespace {
 
-// Scratch of moe_route_topk_noalloc: the control words, the look-back words
-// of the route blocks, the in-expert positions of the picks and a copy of the
-// offsets of one call.  Every GPU that loads this library holds these bytes
-// until the process exits.
+// Scratch of moe_route_topk_noalloc: the control words, the per-block count
+// and base tables and the per-token ranks of one call.  Every GPU that loads
+// this library holds these bytes until the process exits.
 static __device__ __align__(256) unsigned char g_route_scratch[MOE_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
@@ -43,15 +42,16 @@ namespace {
 
 // Byte offsets inside the scratch array for a call with n tokens.
 struct NoallocLayout {
-  size_t flags, pos, off, end;
+  size_t blk, bases, rank, end;
 };
 
 NoallocLayout noalloc_layout(const moe_plan& p, int32_t n) {
+  const size_t table = moe::align256(size_t(moe::route_blocks(n)) * p.d.n_experts * 4);
   NoallocLayout L;
-  L.flags = sizeof(moe::Ctrl);
-  L.pos = L.flags + moe::align256(size_t(moe::route_blocks(n)) * p.d.n_experts * 4);
-  L.off = L.pos + moe::align256(size_t(n) * p.d.top_k * 4);
-  L.end = L.off + moe::align256(size_t(p.d.n_experts + 1) * 4);
+  L.blk = sizeof(moe::Ctrl);
+  L.bases = L.blk + table;
+  L.rank = L.bases + table;
+  L.end = L.rank + moe::align256(size_t(n) * p.d.top_k);
   return L;
 }
 
@@ -77,13 +77,13 @@ extern "C" MOE_API moe_status moe_route_topk_noalloc(const moe_plan* p, int32_t 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   char* b = static_cast<char*>(base);
   // The array keeps whatever the previous call left: the control words
-  // (status, ticket) and this call's look-back words must start at zero.
-  // The positions and offsets are fully rewritten.
-  if (cudaMemsetAsync(b, 0, L.pos, st) != cudaSuccess) return MOE_ERR_CUDA;
+  // (status, the route kernel's counter) must start at zero.  The tables are
+  // fully rewritten.
+  if (cudaMemsetAsync(b, 0, sizeof(moe::Ctrl), st) != cudaSuccess) return MOE_ERR_CUDA;
   const cudaError_t e = moe::launch_route_on(
       *p, n, logits, topk_idx, topk_w, counts, expert_off, b,
-      reinterpret_cast<uint32_t*>(b + L.flags), reinterpret_cast<int32_t*>(b + L.pos),
-      reinterpret_cast<int32_t*>(b + L.off), st);
+      reinterpret_cast<int32_t*>(b + L.blk), reinterpret_cast<int32_t*>(b + L.bases),
+      reinterpret_cast<uint8_t*>(b + L.rank), st);
   if (e == cudaSuccess) return MOE_OK;
   return e == cudaErrorNotSupported ? MOE_ERR_UNSUPPORTED : MOE_ERR_CUDA;
 }

@@ -180,6 +180,11 @@ __global__ void __launch_bounds__(kRThreads, 1)
   const int S = g.split;
   const int m_tile = int(blockIdx.x) / S;
   const int kb0 = int(rank) * g.k_steps;
+  // The m-tiles of the grid read the same router rows; each starts its walk
+  // over its k-blocks at a different one, so that they do not all ask the
+  // same L2 lines for the same bytes at the same moment.  The order is fixed
+  // per tile: the logits do not depend on timing.
+  const int kb_rot = (m_tile * 5) % g.k_steps;
   const uint32_t b_bytes = uint32_t(g.n_mma) * kRBK * 2;
 
   if (threadIdx.x == 0) {
@@ -219,8 +224,9 @@ __global__ void __launch_bounds__(kRThreads, 1)
         }
         uint8_t* a_dst = smem + size_t(stage) * kRStageBytes;
         mbar_arrive_expect_tx(&full[stage], kRABytes + b_bytes);
-        tma_2d(a_dst, &tma_x, (kb0 + kb) * kRBK, m_tile * kRBM, &full[stage]);
-        tma_2d(a_dst + kRABytes, &tma_w, (kb0 + kb) * kRBK, 0, &full[stage]);
+        const int kk = kb0 + (kb + kb_rot) % g.k_steps;
+        tma_2d(a_dst, &tma_x, kk * kRBK, m_tile * kRBM, &full[stage]);
+        tma_2d(a_dst + kRABytes, &tma_w, kk * kRBK, 0, &full[stage]);
         ++issued;
         if (++stage == kRStages) stage = 0, phase ^= 1u;
       }

@@ -114,7 +114,7 @@ typedef struct moe_plan moe_plan;
 
 /* Validate `desc` and build a plan (host only, no CUDA call).
  * Requires: every row (x, Y, out) a multiple of 16 bytes; scale_block > 0
- * only with FP8 rows and dividing D; n_max < 2^30; T(n_max) < 2^31; for inter > 0 also
+ * only with FP8 rows and dividing D; T(n_max) < 2^31; for inter > 0 also
  * y = BF16, D % 256 == 0, I % 128 == 0 and either x = BF16 (bf16 experts) or
  * x = FP8 with scale_block = 128 (FP8 experts).  *out is set only on MOE_OK. */
 MOE_API moe_status moe_plan_create(const moe_desc* desc, moe_plan** out);
@@ -136,12 +136,11 @@ MOE_API int64_t moe_recv_rows(const moe_plan* plan, int32_t n);
  *                        of the same rank;  expert_off[E] = T.
  * logits: device fp32 [n, E] row-major.  topk_idx: device int32 [n, k];
  * topk_w: device fp32 [n, k]; counts: device int32 [E]; expert_off: device
- * int32 [E + 1].  Also leaves in `ws` each pick's position inside its
- * expert's segment and a copy of the offsets, from which moe_dispatch takes
- * the slots of this routing.  n = 0 writes zero counts and offsets.  One
- * launch, no grid-wide barrier: route blocks of 32 tokens take tickets in the
- * order they start and find their prefix of every expert's count by a
- * bounded look-back over the earlier blocks' published counts. */
+ * int32 [E + 1].  Also leaves in `ws` the per-block bases that moe_dispatch
+ * uses for the slots of this routing.  n = 0 writes zero counts and offsets.
+ * One launch in which no block waits for another: each block of 32 tokens
+ * routes them and writes its per-expert counts, and the block that finishes
+ * last scans all blocks' counts into the offsets and per-block bases. */
 MOE_API moe_status moe_route_topk(const moe_plan* plan, int32_t n, const float* logits,
                           int32_t* topk_idx, float* topk_w, int32_t* counts,
                           int32_t* expert_off, void* ws, moe_stream_t stream);
@@ -156,7 +155,7 @@ MOE_API moe_status moe_route_topk(const moe_plan* plan, int32_t n, const float* 
  * x: device bf16 [n, D] hidden rows (with FP8 dispatch rows, the bf16 rows
  * they were quantised from); w_router: device bf16 [E, D]; logits: device
  * fp32 [n, E] or NULL (not written); topk_idx, topk_w, counts, expert_off as
- * in moe_route_topk, and the call leaves the same positions in ws for
+ * in moe_route_topk, and the call leaves the same per-block bases in ws for
  * moe_dispatch.  The selection is exact on the logits this call computes
  * (the same rule as moe_route_topk on them).  Requires D % 64 == 0 and
  * E <= 256 (MOE_ERR_UNSUPPORTED otherwise).  n = 0 writes zero counts and
@@ -170,7 +169,7 @@ MOE_API moe_status moe_router_topk(const moe_plan* plan, int32_t n, const void* 
  * recv_scale[slot(t, j)] = x_scale[t] (D / scale_block fp32, when scale_block
  * > 0), slot_of[t, j] = slot(t, j), src_of[slot(t, j)] = t*k + j.
  * Must follow moe_route_topk on the same stream with the same n, topk_idx and
- * ws (the slots come from that call's positions and offsets).  x: device [n, D];
+ * ws (the slots come from that call's per-block bases).  x: device [n, D];
  * x_scale: device fp32 [n, D/scale_block] or NULL when scale_block == 0;
  * recv: device [T, D]; recv_scale: device fp32 [T, D/scale_block] or NULL;
  * slot_of: device int32 [n, k]; src_of: device int32 [T] (only filled slots
@@ -184,12 +183,10 @@ MOE_API moe_status moe_dispatch(const moe_plan* plan, int32_t n, const void* x, 
  * layouts, same errors).  For n <= 1024 tokens both run in ONE launch: the
  * decode-size step where fixed per-launch costs outweigh the bytes moved (the
  * small-batch regime of "One-Sided Expert-Parallel All-to-All for Mixture-of-
- * Experts Inference over NVLink", abstract).  Up to 256 tokens every block
- * routes all tokens itself from the (L2-resident) logits and scatters its
- * own, with no grid barrier; from 257 to 1024 tokens a cooperative launch in
- * which each block routes and scatters its own tokens, with a single grid
- * barrier between routing and scattering.  Larger n runs the two kernels.  Unlike
- * moe_route_topk, the one-launch form leaves no positions in ws for a
+ * Experts Inference over NVLink", abstract): a cooperative launch in which
+ * each block routes and scatters its own tokens, with a single grid barrier
+ * between routing and scattering.  Larger n runs the two kernels.  Unlike
+ * moe_route_topk, the one-launch form leaves no per-block bases in ws for a
  * later moe_dispatch.  n = 0 writes zero counts and offsets only.  No
  * counterpart call on the pages: it fuses two of their steps. */
 MOE_API moe_status moe_route_dispatch(const moe_plan* plan, int32_t n, const float* logits,
@@ -290,10 +287,9 @@ MOE_API void* moe_layer_buffer(const moe_plan* plan, void* ws, const char* name)
  * (MOE_ERR_CUDA if the copy itself fails). */
 MOE_API moe_status moe_get_status(const moe_plan* plan, void* ws, moe_stream_t stream);
 
-/* Zero the control words, the route kernel's look-back words and the fused
- * kernel's token masks of a workspace (an alternative to zero-filling it),
- * enqueued on `stream`.  Required again after a call reported
- * MOE_ERR_TIMEOUT. */
+/* Zero the control words and the fused kernel's token masks of a workspace
+ * (an alternative to zero-filling it), enqueued on `stream`.  Required again
+ * after a call reported MOE_ERR_TIMEOUT. */
 MOE_API moe_status moe_workspace_init(const moe_plan* plan, void* ws, moe_stream_t stream);
 
 /* Bytes of the fixed scratch array that moe_route_topk_noalloc uses. */
@@ -317,7 +313,7 @@ MOE_API moe_status moe_workspace_init(const moe_plan* plan, void* ws, moe_stream
  * Device-detected errors are recorded in the array, where moe_get_status
  * cannot see them: moe_route_topk_noalloc_status reads them (for the most
  * recent call on the current device; each call starts from MOE_OK).  The
- * positions stay inside the array, so this call's routing cannot feed
+ * per-block tables stay inside the array, so this call's routing cannot feed
  * moe_dispatch.  The array's device address is looked up once per device and
  * kept for the life of the process: after a cudaDeviceReset (or anything
  * else that destroys the device's primary context) it is stale, so do not

@@ -1,8 +1,6 @@
-"""moe_route_dispatch (one launch for n <= 1024 tokens: up to 256 tokens every
-block routes all tokens and scatters its own with no grid barrier, above that a
-cooperative launch in which each block routes and scatters its own tokens
-around one grid barrier) against the CPU oracle and against the two-call path,
-through the C ABI.
+"""moe_route_dispatch (one cooperative launch for n <= 1024 tokens, each block
+routing and scattering its own tokens around one grid barrier) against the CPU
+oracle and against the two-call path, through the C ABI.
 
 The fused call must give exactly what moe_route_topk followed by moe_dispatch
 gives: every integer result and every dispatched byte bit-exact, gate weights
