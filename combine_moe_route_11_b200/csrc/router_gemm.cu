@@ -9,7 +9,8 @@
 // One 128-token tile of x against all E (<= 256) router rows is a single
 // M = 128, N = E MMA chain over K = D.  A tile alone would keep one SM busy
 // for the whole reduction, so the reduction is split over the S CTAs of a
-// thread-block cluster (S = 1, 2, 4 or 8, as many as the grid has room for):
+// thread-block cluster (S = 1, 2, 4 or 8: as many as keep all clusters of
+// the grid resident at once):
 // CTA r of the cluster accumulates k-blocks [r*D/S, (r+1)*D/S) in tensor
 // memory.  Then
 //   1. every CTA copies its 128 x E partial sums from tensor memory into its
@@ -33,6 +34,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <type_traits>
 
 namespace moe {
@@ -180,11 +182,6 @@ __global__ void __launch_bounds__(kRThreads, 1)
   const int S = g.split;
   const int m_tile = int(blockIdx.x) / S;
   const int kb0 = int(rank) * g.k_steps;
-  // The m-tiles of the grid read the same router rows; each starts its walk
-  // over its k-blocks at a different one, so that they do not all ask the
-  // same L2 lines for the same bytes at the same moment.  The order is fixed
-  // per tile: the logits do not depend on timing.
-  const int kb_rot = (m_tile * 5) % g.k_steps;
   const uint32_t b_bytes = uint32_t(g.n_mma) * kRBK * 2;
 
   if (threadIdx.x == 0) {
@@ -224,9 +221,8 @@ __global__ void __launch_bounds__(kRThreads, 1)
         }
         uint8_t* a_dst = smem + size_t(stage) * kRStageBytes;
         mbar_arrive_expect_tx(&full[stage], kRABytes + b_bytes);
-        const int kk = kb0 + (kb + kb_rot) % g.k_steps;
-        tma_2d(a_dst, &tma_x, kk * kRBK, m_tile * kRBM, &full[stage]);
-        tma_2d(a_dst + kRABytes, &tma_w, kk * kRBK, 0, &full[stage]);
+        tma_2d(a_dst, &tma_x, (kb0 + kb) * kRBK, m_tile * kRBM, &full[stage]);
+        tma_2d(a_dst + kRABytes, &tma_w, (kb0 + kb) * kRBK, 0, &full[stage]);
         ++issued;
         if (++stage == kRStages) stage = 0, phase ^= 1u;
       }
@@ -382,12 +378,52 @@ bool router_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Clusters of `split` CTAs of this kernel that can be resident at once.
+int max_active_clusters(const void* kernel, int split) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(split));
+  cfg.blockDim = dim3(kRThreads);
+  cfg.dynamicSmemBytes = kRSmem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = unsigned(split);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess) return 0;
+  return n;
+}
+
 template <int VPL, int VEC>
-cudaError_t launch_router_k(const CUtensorMap& mx, const CUtensorMap& mw, const RouterArgs& g,
-                            int m_tiles, cudaStream_t st) {
+cudaError_t launch_router_k(const CUtensorMap& mx, const CUtensorMap& mw, RouterArgs g,
+                            int m_tiles, int k_total, int sms, cudaStream_t st) {
   auto kernel = router_gemm_kernel<VPL, VEC>;
   cudaError_t e = set_smem_limit(reinterpret_cast<const void*>(kernel), int(kRSmem));
   if (e != cudaSuccess) return e;
+  // Split the reduction over as many CTAs per cluster as keep every cluster
+  // of the grid resident at once (a second wave of clusters would double the
+  // time), up to 8.
+  static std::atomic<int> fits[64][4];  // per device and split 1,2,4,8: resident clusters (0 = unknown)
+  int dev = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if (dev >= 64) return cudaErrorInvalidDevice;
+  int split = 1;
+  for (int lg = 1; lg < 4; ++lg) {
+    const int s = 1 << lg;
+    if (m_tiles * s > sms || k_total % s != 0) break;
+    int c = fits[dev][lg].load(std::memory_order_relaxed);
+    if (c == 0) {
+      c = max_active_clusters(reinterpret_cast<const void*>(kernel), s);
+      if (c <= 0) break;
+      fits[dev][lg].store(c, std::memory_order_relaxed);
+    }
+    if (c < m_tiles) break;
+    split = s;
+  }
+  g.split = split;
+  g.k_steps = k_total / split;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned(m_tiles * g.split));
   cfg.blockDim = dim3(kRThreads);
@@ -443,16 +479,13 @@ cudaError_t launch_router(const moe_plan& p, int32_t n, const void* x, const voi
   const int m_tiles = (n + kRBM - 1) / kRBM;
   const int k_total = D / kRBK;
   const int sms = num_sms();
-  int split = 1;
-  while (split < kRMaxSplit && m_tiles * split * 2 <= sms && k_total % (split * 2) == 0) split *= 2;
-  g.split = split;
-  g.k_steps = k_total / split;
   CUtensorMap mx, mw;
   if (!router_map(&mx, x, uint64_t(n), uint64_t(D), kRBM) ||
       !router_map(&mw, w_router, uint64_t(E), uint64_t(D), uint32_t(g.n_mma)))
     return cudaErrorInvalidValue;
   return with_router_shape(E, [&](auto vpl, auto vec) {
-    return launch_router_k<decltype(vpl)::value, decltype(vec)::value>(mx, mw, g, m_tiles, st);
+    return launch_router_k<decltype(vpl)::value, decltype(vec)::value>(mx, mw, g, m_tiles, k_total,
+                                                                        sms, st);
   });
 }
 

@@ -99,6 +99,8 @@ CASES = [
     ("tiny_e8", C["tiny"].replace(x_dtype="bf16", y_dtype="bf16", out_dtype="bf16"), 200, None),
     # E = 48: neither a multiple of 32 nor of 128
     ("e48_k5", C["decode"].replace(n_experts=48, top_k=5, n_ranks=4, hidden=1024), 257, None),
+    # 18 tiles, the last one ragged, over clusters of 4
+    ("many_tiles_ragged", C["skewed"], 2300, None),
     # k = 1 and k = E
     ("k1", C["decode"].replace(top_k=1, n_ranks=1), 130, None),
     ("k_eq_e", C["decode"].replace(n_experts=16, top_k=16, n_ranks=2, hidden=512), 70, None),
@@ -128,11 +130,12 @@ def test_router_without_logits_output_selects_the_same():
         assert torch.equal(a[key], b[key]), key
 
 
-def test_router_is_deterministic():
+@pytest.mark.parametrize("n", [1024, 4096])
+def test_router_is_deterministic(n):
     """The split-K partial sums are added in cluster-rank order: two calls
-    give the same logits bit for bit."""
+    give the same logits bit for bit (clusters of 8 and of 4)."""
     cfg = C["prefill"]
-    x, w = _inputs(cfg, 1024, seed=4)
+    x, w = _inputs(cfg, n, seed=4)
     a = run_router(cfg, x, w)
     b = run_router(cfg, x, w)
     assert torch.equal(a["logits"], b["logits"])
