@@ -85,12 +85,14 @@ def describe(cfg, n: int) -> str:
 
 
 def step_config(cfg, n: int, n_sets: int, world: int, graph: bool = False,
-                two_kernel: bool = False) -> dict:
+                two_kernel: bool = False, warm: bool = False) -> dict:
     """The `config` object shared by both arms' JSON lines."""
     step_bytes = algorithmic_bytes(cfg, n)["step"]
     return {"workload": describe(cfg, n), "parallelism": f"replicas{world}",
             "launch": "one CUDA graph per step, replayed" if graph else "eager stream launches",
-            "l2": (f"no flush: {n_sets} buffer set(s) rotate so a step's data was last touched "
+            "l2": (f"warm: one buffer set reused by every step ({step_bytes / 1e6:.0f} MB, "
+                   f"{'inside' if step_bytes < L2_BYTES else 'larger than'} the L2)" if warm else
+                   f"no flush: {n_sets} buffer set(s) rotate so a step's data was last touched "
                    f">= 4x L2 ({step_bytes * max(1, n_sets - 1) / 1e6:.0f} MB of traffic) "
                    f"earlier; steps run back to back"),
             "timed": ("moe_route_topk + moe_dispatch + moe_combine: 3 launches/step"
@@ -633,7 +635,7 @@ def run_ours(args, cfg):
     nb = algorithmic_bytes(cfg, n)
     # Buffer sets rotate so that a step never finds its data in L2: the other
     # sets' traffic between two uses of a set is at least 4x the L2 size.
-    n_sets = buffer_sets(cfg, n)
+    n_sets = 1 if args.warm_l2 else buffer_sets(cfg, n)
     sets = []
     for si in range(n_sets):
         inp = workloads.make_inputs(cfg, seed=rank * 1000 + si, n=n)
@@ -779,7 +781,8 @@ def run_ours(args, cfg):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": path_dtype(cfg), "data": "synthetic",
-            "config": step_config(cfg, n, n_sets, world, args.graph, args.two_kernel),
+            "config": step_config(cfg, n, n_sets, world, args.graph, args.two_kernel,
+                                  args.warm_l2),
             "repeats": len(region_ms),
             "region_ms_per_step": percentiles([r / args.steps for r in region_ms]),
             "step_ms": dict(percentiles(per_step), how="one event after every step"),
@@ -1058,6 +1061,9 @@ def main(argv=None):
     ap.add_argument("--two-kernel", action="store_true",
                     help="time the route and dispatch kernels (moe_route_topk + moe_dispatch) "
                          "even where moe_route_dispatch would run them as one launch")
+    ap.add_argument("--warm-l2", action="store_true",
+                    help="reuse one buffer set in every step, so a step that fits in L2 finds "
+                         "its data there (the default rotates sets so that it never does)")
     ap.add_argument("--graph", action="store_true",
                     help="replay each step as one captured CUDA graph")
     ap.add_argument("--tokens", type=int, default=0,

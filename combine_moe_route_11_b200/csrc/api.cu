@@ -68,6 +68,9 @@ Layout make_layout(const moe_plan& p) {
   // kernel's token masks [2, mask rows, E] (alternate halves by its
   // grid-barrier generation)
   L.masks = take(size_t(2) * mask_rows(p) * d.n_experts * 4);
+  // the route kernel's per-expert totals [2, E], also cleared there: a call
+  // adds into one half and clears the other for the next call
+  L.totals = take(size_t(2) * d.n_experts * 4);
   L.blk = take(size_t(p.blocks_max) * d.n_experts * 4);
   L.bases = take(size_t(p.blocks_max) * d.n_experts * 4);
   L.rank = take(size_t(d.n_max) * d.top_k);
@@ -146,6 +149,8 @@ moe_status moe_plan_create(const moe_desc* desc, moe_plan** out) {
   tmp.blocks_max = route_blocks(d.n_max);
   const int64_t T = total_rows(tmp, d.n_max);
   if (T >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
+  // the route kernel indexes its [blocks, E] tables with 32-bit offsets
+  if (int64_t(tmp.blocks_max) * d.n_experts >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
   tmp.total_max = T;
   tmp.lay = make_layout(tmp);
   moe_plan* p = new (std::nothrow) moe_plan(tmp);

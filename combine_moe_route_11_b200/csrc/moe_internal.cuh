@@ -26,8 +26,9 @@ struct Ctrl {
   unsigned int arrive;    // fused kernel's grid barrier: blocks arrived (reset by the last one)
   int status;             // first device-detected error, 0 = none
   unsigned int gen;       // fused kernel's grid barrier: generation, bumped when all arrived
-  unsigned int ticket;    // route kernel: route blocks done (reset by the last one)
-  unsigned int pad[60];
+  unsigned int ticket;    // route kernel: route blocks arrived (reset by the last one)
+  unsigned int rgen;      // route kernel: calls completed; selects the half of the totals
+  unsigned int pad[59];
 };
 static_assert(sizeof(Ctrl) == 256, "control block is 256 bytes");
 
@@ -39,7 +40,7 @@ inline int elem_bytes(int dtype) {
 
 // Byte offsets of every buffer inside a workspace, fixed by n_max.
 struct Layout {
-  size_t ctrl, masks, blk, bases, rank, route_end;  // [ctrl, blk) is cleared by moe_workspace_init
+  size_t ctrl, masks, totals, blk, bases, rank, route_end;  // [ctrl, blk) is cleared by moe_workspace_init
   size_t topk_idx, topk_w, counts, expert_off, slot_of, src_of, recv, recv_scale, y, h;
   size_t hq, h_scale;  // FP8 SwiGLU experts: H in e4m3 and its per-128-column scales
   size_t end;
@@ -81,7 +82,8 @@ cudaError_t launch_route(const moe_plan& p, int32_t n, const float* logits, int3
 // ([n, k] bytes).
 cudaError_t launch_route_on(const moe_plan& p, int32_t n, const float* logits, int32_t* topk_idx,
                             float* topk_w, int32_t* counts, int32_t* expert_off, void* ctrl,
-                            int32_t* blk, int32_t* bases, uint8_t* rank, cudaStream_t st);
+                            int32_t* totals, int32_t* blk, int32_t* bases, uint8_t* rank,
+                            cudaStream_t st);
 cudaError_t launch_route_counts(const moe_plan& p, int32_t n, int32_t* topk_idx, int32_t* counts,
                                 int32_t* expert_off, void* ws, cudaStream_t st);
 cudaError_t launch_router(const moe_plan& p, int32_t n, const void* x, const void* w_router,

@@ -10,7 +10,7 @@
 // ("backends/mlx: runtime MoE expert-sort for decode", author update on the
 // sorted branch) -- computed here as a counting sort, without any sort.
 //
-// One ordinary launch; no block ever waits for another:
+// One ordinary launch:
 //  1. per route block of 32 tokens (one CTA, one warp per token): the k
 //     largest logits by k rounds of a warp argmax on order-preserving integer
 //     keys (two single-instruction warp reductions per round; the lower
@@ -19,14 +19,18 @@
 //     (token, expert) pair its rank among the block's tokens (popcount of the
 //     lower lanes) and the block's count of the expert, written to a
 //     [blocks, E] table;
-//  2. each CTA then counts itself done on a workspace counter; the CTA that
-//     finishes last reads the whole count table at once (every load in
-//     flight together), scans each expert's column over the route blocks,
-//     turns the expert totals into the rank-major offsets and writes each
-//     route block's absolute base slot per expert.
+//  2. each CTA adds its counts into per-expert totals (integer atomics: the
+//     sums do not depend on their order) and then counts itself arrived on a
+//     workspace counter.  The last P = min(blocks, 8) CTAs to arrive share
+//     the base table: each waits (bounded) until the very last one has
+//     arrived, computes the rank-major offsets from the totals, and scans
+//     1/P of the expert columns over the route blocks into absolute base
+//     slots, with all of its column loads in flight together.  At most P - 1
+//     CTAs ever wait, so the others always have SMs to run on.
 // A slot is then base[block][e] + rank.  All integer results are
-// deterministic: no atomic decides an order.  The counter is reset by the
-// CTA that read it last, so the next call finds it at zero.
+// deterministic: no atomic decides an order.  The last arrival resets the
+// counter and bumps a generation word, which selects the half of the
+// double-buffered totals a call adds into (the previous call cleared it).
 #include "route_common.cuh"
 
 #include <type_traits>
@@ -35,51 +39,31 @@ namespace moe {
 namespace {
 
 static_assert(kWarps == 32, "one warp per token of a 32-token route block");
-constexpr int kScanCache = 32;  // count-table rows a scanning thread keeps in registers
+constexpr int kScanCache = 16;  // count-table rows a scanning thread keeps in registers
+constexpr int kScanBatch = 8;  // count-table rows per batch when they are not all cached
+constexpr int kScanners = 8;   // CTAs that share the base table: the last ones to arrive
 
-// The last CTA: column sums of the [B, E] count table, the rank-major
-// offsets, and the absolute base of every (route block, expert).  Thread
-// (e, q) with e = tid % E, q = tid / E (Q = kRouteThreads / E threads per
-// column) owns rows [q * rows_q, (q + 1) * rows_q) of column e.
-__device__ __forceinline__ void scan_counts(const RouteArgs& a, int32_t* s_part, int32_t* s_pre,
-                                            int32_t* s_wsum) {
+// Rows [r, min(r + kScanBatch, r1)) of a count column (zero past r1); the
+// column holds at most blocks * E < 2^31 elements past `col`.
+__device__ __forceinline__ void load_rows(const int32_t* col, int r, int r1, int E,
+                                          int32_t (&v)[kScanBatch]) {
+#pragma unroll
+  for (int i = 0; i < kScanBatch; ++i) v[i] = r + i < r1 ? __ldcg(col + (r + i) * E) : 0;
+}
+
+// One scanning CTA, once every CTA has arrived: the rank-major offsets of all
+// experts from their totals (every scanner computes them; `writer` stores
+// counts and expert_off), then the absolute base of every (route block,
+// expert) for the experts [c0, c1).  Thread (e, q), e in [c0, c1), owns rows
+// [q * rows_q, (q + 1) * rows_q) of column e.
+__device__ __forceinline__ void scan_columns(const RouteArgs& a, const int32_t* tot, int c0,
+                                             int c1, bool writer, int32_t* s_part,
+                                             int32_t* s_pre, int32_t* s_wsum) {
   const int E = a.E, B = a.blocks;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int Q = kRouteThreads / E;  // E <= 512, so Q >= 2
-  const int rows_q = (B + Q - 1) / Q;
-  const bool active = tid < Q * E;
-  const int e = active ? tid % E : 0, q = active ? tid / E : 0;
-  const int r0 = min(B, q * rows_q), r1 = min(B, r0 + rows_q);
-  const int32_t* col = a.blk + e;
-  int32_t* bcol = a.bases + e;
-  // ---- pass 1: this thread's sum of its rows (kept when there are few)
-  int32_t c[kScanCache];
-  int sum = 0;
-  const bool cached = rows_q <= kScanCache;
-  if (active) {
-    if (cached) {
-#pragma unroll
-      for (int i = 0; i < kScanCache; ++i)
-        c[i] = r0 + i < r1 ? __ldcg(col + int64_t(r0 + i) * E) : 0;
-#pragma unroll
-      for (int i = 0; i < kScanCache; ++i) sum += c[i];
-    } else {
-      for (int r = r0; r < r1; r += 16) {
-        int32_t v[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = r + i < r1 ? __ldcg(col + int64_t(r + i) * E) : 0;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) sum += v[i];
-      }
-    }
-    s_part[q * E + e] = sum;
-  }
-  __syncthreads();
-  // ---- expert totals and their exclusive prefix over all experts
-  int tot = 0;
-  if (tid < E)
-    for (int q2 = 0; q2 < Q; ++q2) tot += s_part[q2 * E + tid];
-  int incl = tot;
+  // ---- offsets of all experts: exclusive prefix of the totals
+  const int t_e = tid < E ? __ldcg(tot + tid) : 0;
+  int incl = t_e;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const int y = __shfl_up_sync(kFull, incl, o);
@@ -98,40 +82,79 @@ __device__ __forceinline__ void scan_counts(const RouteArgs& a, int32_t* s_part,
     s_wsum[lane] = wi - w;
   }
   __syncthreads();
-  const int pre = incl - tot + s_wsum[warp];
+  const int pre = incl - t_e + s_wsum[warp];
   if (tid < E) s_pre[tid] = pre;
   __syncthreads();
   const int per_rank = E / a.R;
-  if (tid < E) {
+  if (writer && tid < E) {
     const int r = tid / per_rank;
-    const int off = r * a.region_rows + pre - s_pre[r * per_rank];
-    a.counts[tid] = tot;
-    a.expert_off[tid] = off;
+    a.counts[tid] = t_e;
+    a.expert_off[tid] = r * a.region_rows + pre - s_pre[r * per_rank];
   }
-  if (tid == 0) a.expert_off[E] = a.R * a.region_rows;
-  // ---- pass 2: absolute bases of this thread's rows
+  if (writer && tid == 0) a.expert_off[E] = a.R * a.region_rows;
+  // ---- this scanner's columns
+  const int ncol = c1 - c0;
+  if (ncol <= 0) return;
+  const int Q = kRouteThreads / ncol;  // threads per column (ncol <= 512, so Q >= 2)
+  const int rows_q = (B + Q - 1) / Q;
+  const bool active = tid < Q * ncol;
+  const int e = c0 + (active ? tid % ncol : 0), q = active ? tid / ncol : 0;
+  const int r0 = min(B, q * rows_q), r1 = min(B, r0 + rows_q);
+  // this thread's rows of the count column and of the base column
+  const int32_t* col = a.blk + int64_t(r0) * E + e;
+  int32_t* bcol = a.bases + int64_t(r0) * E + e;
+  const int nr = r1 - r0;
+  // pass 1: this thread's sum of its rows (kept when there are few)
+  int32_t c[kScanCache];
+  int sum = 0;
+  const bool cached = rows_q <= kScanCache;
+  if (active) {
+    if (cached) {
+#pragma unroll
+      for (int i = 0; i < kScanCache; ++i) c[i] = i < nr ? __ldcg(col + i * E) : 0;
+#pragma unroll
+      for (int i = 0; i < kScanCache; ++i) sum += c[i];
+    } else {
+      int32_t v[kScanBatch];
+      load_rows(col, 0, nr, E, v);
+      for (int r = 0; r < nr; r += kScanBatch) {
+        int32_t w[kScanBatch];
+        load_rows(col, r + kScanBatch, nr, E, w);
+#pragma unroll
+        for (int i = 0; i < kScanBatch; ++i) sum += v[i];
+#pragma unroll
+        for (int i = 0; i < kScanBatch; ++i) v[i] = w[i];
+      }
+    }
+    s_part[q * ncol + (e - c0)] = sum;
+  }
+  __syncthreads();
+  // pass 2: absolute bases of this thread's rows
   if (active) {
     const int rk = e / per_rank;
     int run = rk * a.region_rows + s_pre[e] - s_pre[rk * per_rank];
-    for (int q2 = 0; q2 < q; ++q2) run += s_part[q2 * E + e];
+    for (int q2 = 0; q2 < q; ++q2) run += s_part[q2 * ncol + (e - c0)];
     if (cached) {
 #pragma unroll
       for (int i = 0; i < kScanCache; ++i)
-        if (r0 + i < r1) {
-          bcol[int64_t(r0 + i) * E] = run;
+        if (i < nr) {
+          bcol[i * E] = run;
           run += c[i];
         }
     } else {
-      for (int r = r0; r < r1; r += 16) {
-        int32_t v[16];
+      int32_t v[kScanBatch];
+      load_rows(col, 0, nr, E, v);
+      for (int r = 0; r < nr; r += kScanBatch) {
+        int32_t w[kScanBatch];
+        load_rows(col, r + kScanBatch, nr, E, w);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = r + i < r1 ? __ldcg(col + int64_t(r + i) * E) : 0;
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          if (r + i < r1) {
-            bcol[int64_t(r + i) * E] = run;
+        for (int i = 0; i < kScanBatch; ++i)
+          if (r + i < nr) {
+            bcol[(r + i) * E] = run;
             run += v[i];
           }
+#pragma unroll
+        for (int i = 0; i < kScanBatch; ++i) v[i] = w[i];
       }
     }
   }
@@ -144,21 +167,27 @@ template <int VPL, int VEC, bool kFromIdx>
 __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(RouteArgs a) {
   __shared__ int32_t s_sel[kRouteTokens * kMaxTopK];  // picks of the block's tokens
   __shared__ uint32_t s_mask[kMaxExperts];            // token mask per expert
-  __shared__ int32_t s_part[kRouteThreads];           // last CTA: partial column sums
+  __shared__ int32_t s_part[kRouteThreads];           // scanners: partial column sums
   __shared__ int32_t s_pre[kMaxExperts];
   __shared__ int32_t s_wsum[kWarps];
-  __shared__ int s_last;
+  __shared__ int s_arrival;
+  __shared__ unsigned s_gen;
+  __shared__ int s_ok;
   const int E = a.E, K = a.K, B = a.blocks;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int b = blockIdx.x;
   const int t_base = b * kRouteTokens;
   const int valid = max(0, min(kRouteTokens, a.n - t_base));
+  Ctrl* ctrl = reinterpret_cast<Ctrl*>(a.ws);
   grid_dependency_wait();
+  // the generation of this call: it selects the half of the totals, and the
+  // last arrival bumps it once every CTA has read it
+  if (tid == 0) s_gen = ld_acquire_gpu(&ctrl->rgen);
   for (int i = tid; i < E; i += kRouteThreads) s_mask[i] = 0u;
+  __syncthreads();
 
   // ---- 1. top-k and softmax (one warp per token), or the given picks
   if constexpr (kFromIdx) {
-    __syncthreads();
     for (int p = tid; p < valid * K; p += kRouteThreads) {
       int e = __ldg(a.topk_idx + int64_t(t_base) * K + p);
       if (e < 0 || e >= E) {
@@ -182,7 +211,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(RouteArgs a) {
     }
   }
   __syncthreads();
-  // ---- per-expert token masks, in-block ranks, block counts
+  // ---- per-expert token masks, in-block ranks, block counts, expert totals
   for (int p = tid; p < valid * K; p += kRouteThreads)
     if (!kFromIdx || s_sel[p] >= 0) atomicOr(&s_mask[s_sel[p]], 1u << (p / K));
   __syncthreads();
@@ -191,21 +220,51 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(RouteArgs a) {
     a.rank[int64_t(t_base) * K + p] =
         kFromIdx && e < 0 ? uint8_t(0) : uint8_t(__popc(s_mask[e] & ((1u << (p / K)) - 1u)));
   }
-  for (int e = tid; e < E; e += kRouteThreads) a.blk[int64_t(b) * E + e] = __popc(s_mask[e]);
+  const unsigned gen = s_gen;
+  int32_t* tot = a.totals + size_t(gen & 1u) * E;
+  if (b == 0)  // the other half starts the next call at zero
+    for (int i = tid; i < E; i += kRouteThreads) a.totals[size_t((gen & 1u) ^ 1u) * E + i] = 0;
+  for (int e = tid; e < E; e += kRouteThreads) {
+    const int cnt = __popc(s_mask[e]);
+    a.blk[int64_t(b) * E + e] = cnt;
+    if (cnt) atomicAdd(tot + e, cnt);  // integer sums: the order does not matter
+  }
 
-  // ---- 2. the CTA that finishes last scans the count table
+  // ---- 2. arrival; the last P CTAs to arrive build the base table together
+  const int P = min(B, kScanners);
   __syncthreads();
   if (tid == 0) {
-    Ctrl* ctrl = reinterpret_cast<Ctrl*>(a.ws);
-    fence_acq_rel_gpu();  // this CTA's counts before its arrival
-    s_last = atomicAdd(&ctrl->ticket, 1u) == unsigned(B - 1);
-    if (s_last) {
-      fence_acq_rel_gpu();  // every other CTA's counts before the reads below
-      ctrl->ticket = 0u;    // every CTA has arrived: the next call starts at zero
+    fence_acq_rel_gpu();  // this CTA's counts and totals before its arrival
+    const int arrival = int(atomicAdd(&ctrl->ticket, 1u));
+    int ok = 1;
+    if (arrival == B - 1) {
+      // every CTA has arrived: reset the counter, publish the new generation
+      st_relaxed_gpu(&ctrl->ticket, 0u);
+      fence_acq_rel_gpu();
+      atomicAdd(&ctrl->rgen, 1u);
+    } else if (arrival >= B - P) {
+      // a scanner: wait (bounded) until the last CTA has arrived
+      const long long t0 = clock64();
+      while (ld_acquire_gpu(&ctrl->rgen) == gen) {
+        if (clock64() - t0 > (1ll << 31)) {
+          set_status(a.ws, MOE_ERR_TIMEOUT);
+          ok = 0;
+          break;
+        }
+      }
     }
+    fence_acq_rel_gpu();  // every CTA's counts and totals before the reads below
+    s_arrival = arrival;
+    s_ok = ok;
   }
   __syncthreads();
-  if (s_last) scan_counts(a, s_part, s_pre, s_wsum);
+  const int arrival = s_arrival;
+  if (arrival >= B - P && s_ok) {
+    const int s_idx = arrival - (B - P);
+    const int per = (E + P - 1) / P;
+    scan_columns(a, tot, min(E, s_idx * per), min(E, (s_idx + 1) * per), s_idx == P - 1, s_part,
+                 s_pre, s_wsum);
+  }
   grid_dependents_launch();
 }
 
@@ -237,6 +296,7 @@ RouteArgs ws_args(const moe_plan& p, void* ws) {
   a.blk = reinterpret_cast<int32_t*>(w + p.lay.blk);
   a.bases = reinterpret_cast<int32_t*>(w + p.lay.bases);
   a.rank = reinterpret_cast<uint8_t*>(w + p.lay.rank);
+  a.totals = reinterpret_cast<int32_t*>(w + p.lay.totals);
   a.ws = ws;
   return a;
 }
@@ -270,7 +330,8 @@ cudaError_t launch_route_counts(const moe_plan& p, int32_t n, int32_t* topk_idx,
 
 cudaError_t launch_route_on(const moe_plan& p, int32_t n, const float* logits, int32_t* topk_idx,
                             float* topk_w, int32_t* counts, int32_t* expert_off, void* ctrl,
-                            int32_t* blk, int32_t* bases, uint8_t* rank, cudaStream_t st) {
+                            int32_t* totals, int32_t* blk, int32_t* bases, uint8_t* rank,
+                            cudaStream_t st) {
   RouteArgs a;
   a.logits = logits;
   a.topk_idx = topk_idx;
@@ -280,6 +341,7 @@ cudaError_t launch_route_on(const moe_plan& p, int32_t n, const float* logits, i
   a.blk = blk;
   a.bases = bases;
   a.rank = rank;
+  a.totals = totals;
   a.ws = ctrl;
   return launch_with(a, p, n, st);
 }

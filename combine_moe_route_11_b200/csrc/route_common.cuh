@@ -22,6 +22,7 @@ struct RouteArgs {
   int32_t* blk;    // [blocks, E] per-block counts
   int32_t* bases;  // [blocks, E] per-block absolute base slots
   uint8_t* rank;   // [n, k]: rank of (t, j) among the block's tokens picking e
+  int32_t* totals; // [2, E] per-expert totals, alternate halves per call (route kernel)
   uint32_t* masks; // [2, mask_rows, E] token masks of the fused kernel (null: none)
   int32_t mask_rows;
   void* ws;

@@ -243,6 +243,7 @@ cudaError_t launch_route_dispatch(const moe_plan& p, int32_t n, const float* log
   a.blk = nullptr;
   a.bases = nullptr;
   a.rank = nullptr;
+  a.totals = nullptr;
   a.masks = reinterpret_cast<uint32_t*>(w + p.lay.masks);
   a.mask_rows = mask_rows(p);
   a.ws = ws;

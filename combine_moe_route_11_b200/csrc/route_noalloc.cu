@@ -42,13 +42,14 @@ namespace {
 
 // Byte offsets inside the scratch array for a call with n tokens.
 struct NoallocLayout {
-  size_t blk, bases, rank, end;
+  size_t totals, blk, bases, rank, end;
 };
 
 NoallocLayout noalloc_layout(const moe_plan& p, int32_t n) {
   const size_t table = moe::align256(size_t(moe::route_blocks(n)) * p.d.n_experts * 4);
   NoallocLayout L;
-  L.blk = sizeof(moe::Ctrl);
+  L.totals = sizeof(moe::Ctrl);
+  L.blk = L.totals + moe::align256(size_t(2) * p.d.n_experts * 4);
   L.bases = L.blk + table;
   L.rank = L.bases + table;
   L.end = L.rank + moe::align256(size_t(n) * p.d.top_k);
@@ -77,12 +78,12 @@ extern "C" MOE_API moe_status moe_route_topk_noalloc(const moe_plan* p, int32_t 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   char* b = static_cast<char*>(base);
   // The array keeps whatever the previous call left: the control words
-  // (status, the route kernel's counter) must start at zero.  The tables are
-  // fully rewritten.
-  if (cudaMemsetAsync(b, 0, sizeof(moe::Ctrl), st) != cudaSuccess) return MOE_ERR_CUDA;
+  // (status, the route kernel's counter and generation) and the expert
+  // totals must start at zero.  The tables are fully rewritten.
+  if (cudaMemsetAsync(b, 0, L.blk, st) != cudaSuccess) return MOE_ERR_CUDA;
   const cudaError_t e = moe::launch_route_on(
       *p, n, logits, topk_idx, topk_w, counts, expert_off, b,
-      reinterpret_cast<int32_t*>(b + L.blk), reinterpret_cast<int32_t*>(b + L.bases),
+      reinterpret_cast<int32_t*>(b + L.totals), reinterpret_cast<int32_t*>(b + L.blk), reinterpret_cast<int32_t*>(b + L.bases),
       reinterpret_cast<uint8_t*>(b + L.rank), st);
   if (e == cudaSuccess) return MOE_OK;
   return e == cudaErrorNotSupported ? MOE_ERR_UNSUPPORTED : MOE_ERR_CUDA;

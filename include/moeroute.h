@@ -114,7 +114,8 @@ typedef struct moe_plan moe_plan;
 
 /* Validate `desc` and build a plan (host only, no CUDA call).
  * Requires: every row (x, Y, out) a multiple of 16 bytes; scale_block > 0
- * only with FP8 rows and dividing D; T(n_max) < 2^31; for inter > 0 also
+ * only with FP8 rows and dividing D; T(n_max) < 2^31 and
+ * ceil(n_max / 32) * E < 2^31; for inter > 0 also
  * y = BF16, D % 256 == 0, I % 128 == 0 and either x = BF16 (bf16 experts) or
  * x = FP8 with scale_block = 128 (FP8 experts).  *out is set only on MOE_OK. */
 MOE_API moe_status moe_plan_create(const moe_desc* desc, moe_plan** out);
@@ -138,9 +139,11 @@ MOE_API int64_t moe_recv_rows(const moe_plan* plan, int32_t n);
  * topk_w: device fp32 [n, k]; counts: device int32 [E]; expert_off: device
  * int32 [E + 1].  Also leaves in `ws` the per-block bases that moe_dispatch
  * uses for the slots of this routing.  n = 0 writes zero counts and offsets.
- * One launch in which no block waits for another: each block of 32 tokens
- * routes them and writes its per-expert counts, and the block that finishes
- * last scans all blocks' counts into the offsets and per-block bases. */
+ * One launch: each block of 32 tokens routes them, writes its per-expert
+ * counts and adds them into per-expert totals in `ws`; the last min(blocks,
+ * 8) blocks to finish share the scan of all blocks' counts into the offsets
+ * and per-block bases (each waits, bounded, only for the others to finish;
+ * MOE_ERR_TIMEOUT in the status word if that wait ever ran out). */
 MOE_API moe_status moe_route_topk(const moe_plan* plan, int32_t n, const float* logits,
                           int32_t* topk_idx, float* topk_w, int32_t* counts,
                           int32_t* expert_off, void* ws, moe_stream_t stream);
@@ -287,9 +290,10 @@ MOE_API void* moe_layer_buffer(const moe_plan* plan, void* ws, const char* name)
  * (MOE_ERR_CUDA if the copy itself fails). */
 MOE_API moe_status moe_get_status(const moe_plan* plan, void* ws, moe_stream_t stream);
 
-/* Zero the control words and the fused kernel's token masks of a workspace
- * (an alternative to zero-filling it), enqueued on `stream`.  Required again
- * after a call reported MOE_ERR_TIMEOUT. */
+/* Zero the control words, the route kernel's expert totals and the fused
+ * kernel's token masks of a workspace (an alternative to zero-filling it),
+ * enqueued on `stream`.  Required again after a call reported
+ * MOE_ERR_TIMEOUT or a launch in the workspace's stream failed. */
 MOE_API moe_status moe_workspace_init(const moe_plan* plan, void* ws, moe_stream_t stream);
 
 /* Bytes of the fixed scratch array that moe_route_topk_noalloc uses. */
