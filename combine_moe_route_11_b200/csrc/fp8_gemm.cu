@@ -330,21 +330,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      int stage = 0, buf = 0;
-      uint32_t phase = 0, buf_phase = 0;
-      const uint32_t idesc = idesc_e4m3(kBN);
-      bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        for (int kb = 0; kb < g.k_steps; ++kb) {
-          if (*s_abort || !mbar_wait_hot(&pempty[buf], buf_phase ^ 1u) ||
-              !mbar_wait_hot(&full[stage], phase)) {
-            if (!*s_abort) set_status(g.ws, MOE_ERR_TIMEOUT);
-            *s_abort = 1;
-            ok = false;
-            break;
-          }
-          tc_fence_after();
+    // The whole warp runs the loop and waits; one lane issues.
+    int stage = 0, buf = 0;
+    uint32_t phase = 0, buf_phase = 0;
+    const uint32_t idesc = idesc_e4m3(kBN);
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      for (int kb = 0; kb < g.k_steps; ++kb) {
+        bool w = !*s_abort;
+        if (w) w = mbar_wait_hot(&full[stage], phase);
+        if (w) w = mbar_wait_hot(&pempty[buf], buf_phase ^ 1u);
+        w = __all_sync(0xFFFFFFFFu, w);
+        if (!w) {
+          if (lane == 0 && !*s_abort) set_status(g.ws, MOE_ERR_TIMEOUT);
+          __syncwarp();
+          *s_abort = 1;
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
           const uint32_t d_tmem = tmem_base + uint32_t(buf * kBN);
           const uint32_t a_addr = smem_addr(smem + size_t(stage) * kStageBytes);
           const uint32_t b_addr = a_addr + kABytes;
@@ -354,14 +359,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                       smem_desc_sw128(b_addr + k * kUmmaK), idesc, k != 0 ? 1u : 0u);
           umma_commit(&empty[stage]);  // stage free once these MMAs have read it
           umma_commit(&pfull[buf]);    // partial sum of this k-block ready
-          if (++stage == kStages) stage = 0, phase ^= 1u;
-          if (++buf == 2) buf = 0, buf_phase ^= 1u;
         }
+        __syncwarp();
+        if (++stage == kStages) stage = 0, phase ^= 1u;
+        if (++buf == 2) buf = 0, buf_phase ^= 1u;
       }
-      // every MMA this thread issued has completed before the memory is freed
+    }
+    // every MMA this warp issued has completed before the memory is freed
+    if (lane == 0) {
       umma_commit(drained);
       if (!mbar_wait(drained, 0)) set_status(g.ws, MOE_ERR_TIMEOUT);
     }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ promotion + epilogue
     const int quarter = warp & 3;           // TMEM lanes this warp may read

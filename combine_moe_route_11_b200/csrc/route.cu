@@ -10,8 +10,9 @@
 // ("backends/mlx: runtime MoE expert-sort for decode", author update on the
 // sorted branch) -- computed here as a counting sort, without any sort.
 //
-// One ordinary launch:
-//  1. per route block of 32 tokens (one CTA, one warp per token): the k
+// One ordinary launch of min(blocks, SMs) CTAs, each taking every G-th route
+// block:
+//  1. per route block of 32 tokens (one warp per token): the k
 //     largest logits by k rounds of a warp argmax on order-preserving integer
 //     keys (two single-instruction warp reductions per round; the lower
 //     expert id wins a tie) and a softmax over the k winners; then, per
@@ -20,13 +21,14 @@
 //     lower lanes) and the block's count of the expert, written to a
 //     [blocks, E] table;
 //  2. each CTA adds its counts into per-expert totals (integer atomics: the
-//     sums do not depend on their order) and then counts itself arrived on a
-//     workspace counter.  The last P = min(blocks, 8) CTAs to arrive share
-//     the base table: each waits (bounded) until the very last one has
-//     arrived, computes the rank-major offsets from the totals, and scans
-//     1/P of the expert columns over the route blocks into absolute base
-//     slots, with all of its column loads in flight together.  At most P - 1
-//     CTAs ever wait, so the others always have SMs to run on.
+//     sums do not depend on their order) and, after its last route block,
+//     counts itself arrived on a workspace counter.  The last P = min(CTAs,
+//     8) to arrive share the base table: each waits (bounded) until the very
+//     last one has arrived, computes the rank-major offsets from the totals,
+//     and scans 1/P of the expert columns over the route blocks into
+//     absolute base slots, with all of its column loads in flight together.
+//     Only CTAs that have finished their own blocks wait, at most P - 1 of
+//     them, so the others always have SMs to run on.
 // A slot is then base[block][e] + rank.  All integer results are
 // deterministic: no atomic decides an order.  The last arrival resets the
 // counter and bumps a generation word, which selects the half of the
@@ -173,76 +175,78 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(RouteArgs a) {
   __shared__ int s_arrival;
   __shared__ unsigned s_gen;
   __shared__ int s_ok;
-  const int E = a.E, K = a.K, B = a.blocks;
+  const int E = a.E, K = a.K;
+  const int G = gridDim.x;  // CTAs; each takes route blocks blockIdx.x, + G, + 2G, ...
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int b = blockIdx.x;
-  const int t_base = b * kRouteTokens;
-  const int valid = max(0, min(kRouteTokens, a.n - t_base));
   Ctrl* ctrl = reinterpret_cast<Ctrl*>(a.ws);
   grid_dependency_wait();
   // the generation of this call: it selects the half of the totals, and the
   // last arrival bumps it once every CTA has read it
   if (tid == 0) s_gen = ld_acquire_gpu(&ctrl->rgen);
-  for (int i = tid; i < E; i += kRouteThreads) s_mask[i] = 0u;
   __syncthreads();
-
-  // ---- 1. top-k and softmax (one warp per token), or the given picks
-  if constexpr (kFromIdx) {
-    for (int p = tid; p < valid * K; p += kRouteThreads) {
-      int e = __ldg(a.topk_idx + int64_t(t_base) * K + p);
-      if (e < 0 || e >= E) {
-        set_status(a.ws, MOE_ERR_DEVICE_INDEX);
-        e = -1;
-      }
-      s_sel[p] = e;
-    }
-  } else {
-    if (warp < valid) {
-      float w;
-      bool nonfinite;
-      const int64_t t = int64_t(t_base) + warp;
-      const int e = route_row<VPL, VEC, true>(a.logits + t * E, E, K, lane, &w, &nonfinite);
-      if (lane < K) {
-        a.topk_idx[t * K + lane] = e;
-        a.topk_w[t * K + lane] = w;
-        s_sel[warp * K + lane] = e;
-      }
-      if (nonfinite && lane == 0) set_status(a.ws, MOE_ERR_NONFINITE);
-    }
-  }
-  __syncthreads();
-  // ---- per-expert token masks, in-block ranks, block counts, expert totals
-  for (int p = tid; p < valid * K; p += kRouteThreads)
-    if (!kFromIdx || s_sel[p] >= 0) atomicOr(&s_mask[s_sel[p]], 1u << (p / K));
-  __syncthreads();
-  for (int p = tid; p < valid * K; p += kRouteThreads) {
-    const int e = s_sel[p];
-    a.rank[int64_t(t_base) * K + p] =
-        kFromIdx && e < 0 ? uint8_t(0) : uint8_t(__popc(s_mask[e] & ((1u << (p / K)) - 1u)));
-  }
   const unsigned gen = s_gen;
   int32_t* tot = a.totals + size_t(gen & 1u) * E;
-  if (b == 0)  // the other half starts the next call at zero
+  if (blockIdx.x == 0)  // the other half starts the next call at zero
     for (int i = tid; i < E; i += kRouteThreads) a.totals[size_t((gen & 1u) ^ 1u) * E + i] = 0;
-  for (int e = tid; e < E; e += kRouteThreads) {
-    const int cnt = __popc(s_mask[e]);
-    a.blk[int64_t(b) * E + e] = cnt;
-    if (cnt) atomicAdd(tot + e, cnt);  // integer sums: the order does not matter
+
+  for (int b = blockIdx.x; b < a.blocks; b += G) {
+    const int t_base = b * kRouteTokens;
+    const int valid = max(0, min(kRouteTokens, a.n - t_base));
+    for (int i = tid; i < E; i += kRouteThreads) s_mask[i] = 0u;
+    // ---- 1. top-k and softmax (one warp per token), or the given picks
+    if constexpr (kFromIdx) {
+      for (int p = tid; p < valid * K; p += kRouteThreads) {
+        int e = __ldg(a.topk_idx + int64_t(t_base) * K + p);
+        if (e < 0 || e >= E) {
+          set_status(a.ws, MOE_ERR_DEVICE_INDEX);
+          e = -1;
+        }
+        s_sel[p] = e;
+      }
+    } else {
+      if (warp < valid) {
+        float w;
+        bool nonfinite;
+        const int64_t t = int64_t(t_base) + warp;
+        const int e = route_row<VPL, VEC, true>(a.logits + t * E, E, K, lane, &w, &nonfinite);
+        if (lane < K) {
+          a.topk_idx[t * K + lane] = e;
+          a.topk_w[t * K + lane] = w;
+          s_sel[warp * K + lane] = e;
+        }
+        if (nonfinite && lane == 0) set_status(a.ws, MOE_ERR_NONFINITE);
+      }
+    }
+    __syncthreads();
+    // ---- per-expert token masks, in-block ranks, block counts, expert totals
+    for (int p = tid; p < valid * K; p += kRouteThreads)
+      if (!kFromIdx || s_sel[p] >= 0) atomicOr(&s_mask[s_sel[p]], 1u << (p / K));
+    __syncthreads();
+    for (int p = tid; p < valid * K; p += kRouteThreads) {
+      const int e = s_sel[p];
+      a.rank[int64_t(t_base) * K + p] =
+          kFromIdx && e < 0 ? uint8_t(0) : uint8_t(__popc(s_mask[e] & ((1u << (p / K)) - 1u)));
+    }
+    for (int e = tid; e < E; e += kRouteThreads) {
+      const int cnt = __popc(s_mask[e]);
+      a.blk[int64_t(b) * E + e] = cnt;
+      if (cnt) atomicAdd(tot + e, cnt);  // integer sums: the order does not matter
+    }
+    __syncthreads();  // s_sel and s_mask are reused by the next route block
   }
 
   // ---- 2. arrival; the last P CTAs to arrive build the base table together
-  const int P = min(B, kScanners);
-  __syncthreads();
+  const int P = min(G, kScanners);
   if (tid == 0) {
     fence_acq_rel_gpu();  // this CTA's counts and totals before its arrival
     const int arrival = int(atomicAdd(&ctrl->ticket, 1u));
     int ok = 1;
-    if (arrival == B - 1) {
+    if (arrival == G - 1) {
       // every CTA has arrived: reset the counter, publish the new generation
       st_relaxed_gpu(&ctrl->ticket, 0u);
       fence_acq_rel_gpu();
       atomicAdd(&ctrl->rgen, 1u);
-    } else if (arrival >= B - P) {
+    } else if (arrival >= G - P) {
       // a scanner: wait (bounded) until the last CTA has arrived
       const long long t0 = clock64();
       while (ld_acquire_gpu(&ctrl->rgen) == gen) {
@@ -259,8 +263,8 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(RouteArgs a) {
   }
   __syncthreads();
   const int arrival = s_arrival;
-  if (arrival >= B - P && s_ok) {
-    const int s_idx = arrival - (B - P);
+  if (arrival >= G - P && s_ok) {
+    const int s_idx = arrival - (G - P);
     const int per = (E + P - 1) / P;
     scan_columns(a, tot, min(E, s_idx * per), min(E, (s_idx + 1) * per), s_idx == P - 1, s_part,
                  s_pre, s_wsum);
@@ -268,10 +272,14 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(RouteArgs a) {
   grid_dependents_launch();
 }
 
+// One CTA per SM at most (a CTA of 1024 threads fills an SM): with more route
+// blocks than SMs each CTA takes several, so no block waits for a second
+// wave of CTAs to start.
 template <int VPL, int VEC, bool kFromIdx>
 cudaError_t launch_rk(const RouteArgs& a, cudaStream_t st) {
-  return launch_pdl(route_kernel<VPL, VEC, kFromIdx>, dim3(unsigned(a.blocks)),
-                    dim3(kRouteThreads), 0, st, a);
+  const int grid = a.blocks < num_sms() ? a.blocks : num_sms();
+  return launch_pdl(route_kernel<VPL, VEC, kFromIdx>, dim3(unsigned(grid)), dim3(kRouteThreads),
+                    0, st, a);
 }
 
 cudaError_t launch_with(RouteArgs& a, const moe_plan& p, int32_t n, cudaStream_t st,

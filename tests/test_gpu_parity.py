@@ -38,6 +38,9 @@ SMALL_CASES = [
                           y_dtype="bf16", out_dtype="bf16"), 130),
     ("many_blocks", TINY.replace(n_experts=64, top_k=6, n_ranks=4, hidden=32, x_dtype="bf16",
                                  y_dtype="bf16", out_dtype="f32"), 5000),
+    # four to five route blocks per CTA of the route kernel, the last one ragged
+    ("blocks_per_cta", TINY.replace(n_experts=128, top_k=4, n_ranks=4, hidden=32,
+                                    x_dtype="bf16", y_dtype="bf16", out_dtype="f32"), 20011),
     ("bf16_to_f32", C["decode"].replace(hidden=512, out_dtype="f32"), 77),
     ("fp8_small_D", C["prefill"].replace(hidden=256, n_experts=16, top_k=4, n_ranks=4), 129),
     ("k16", TINY.replace(n_experts=32, top_k=16, n_ranks=2, hidden=64), 100),
