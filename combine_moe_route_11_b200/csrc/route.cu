@@ -63,46 +63,16 @@ __device__ __forceinline__ void scan_columns(const RouteArgs& a, const int32_t* 
                                              int32_t* s_pre, int32_t* s_wsum) {
   const int E = a.E, B = a.blocks;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // ---- offsets of all experts: exclusive prefix of the totals
+  // the totals and this thread's count rows are loaded together: neither
+  // waits for the other
   const int t_e = tid < E ? __ldcg(tot + tid) : 0;
-  int incl = t_e;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(kFull, incl, o);
-    if (lane >= o) incl += y;
-  }
-  if (lane == 31) s_wsum[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    const int w = s_wsum[lane];
-    int wi = w;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(kFull, wi, o);
-      if (lane >= o) wi += y;
-    }
-    s_wsum[lane] = wi - w;
-  }
-  __syncthreads();
-  const int pre = incl - t_e + s_wsum[warp];
-  if (tid < E) s_pre[tid] = pre;
-  __syncthreads();
-  const int per_rank = E / a.R;
-  if (writer && tid < E) {
-    const int r = tid / per_rank;
-    a.counts[tid] = t_e;
-    a.expert_off[tid] = r * a.region_rows + pre - s_pre[r * per_rank];
-  }
-  if (writer && tid == 0) a.expert_off[E] = a.R * a.region_rows;
-  // ---- this scanner's columns
-  const int ncol = c1 - c0;
-  if (ncol <= 0) return;
-  const int Q = kRouteThreads / ncol;  // threads per column (ncol <= 512, so Q >= 2)
-  const int rows_q = (B + Q - 1) / Q;
+  // ---- this scanner's columns: thread (e, q) and its rows
+  const int ncol = max(0, c1 - c0);
+  const int Q = ncol > 0 ? kRouteThreads / ncol : 0;  // threads per column (Q >= 2)
+  const int rows_q = ncol > 0 ? (B + Q - 1) / Q : 0;
   const bool active = tid < Q * ncol;
   const int e = c0 + (active ? tid % ncol : 0), q = active ? tid / ncol : 0;
   const int r0 = min(B, q * rows_q), r1 = min(B, r0 + rows_q);
-  // this thread's rows of the count column and of the base column
   const int32_t* col = a.blk + int64_t(r0) * E + e;
   int32_t* bcol = a.bases + int64_t(r0) * E + e;
   const int nr = r1 - r0;
@@ -130,7 +100,36 @@ __device__ __forceinline__ void scan_columns(const RouteArgs& a, const int32_t* 
     }
     s_part[q * ncol + (e - c0)] = sum;
   }
+  // ---- offsets of all experts: exclusive prefix of the totals
+  int incl = t_e;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(kFull, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) s_wsum[warp] = incl;
   __syncthreads();
+  if (warp == 0) {
+    const int w = s_wsum[lane];
+    int wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(kFull, wi, o);
+      if (lane >= o) wi += y;
+    }
+    s_wsum[lane] = wi - w;
+  }
+  __syncthreads();
+  const int pre = incl - t_e + s_wsum[warp];
+  if (tid < E) s_pre[tid] = pre;
+  __syncthreads();  // also publishes s_part
+  const int per_rank = E / a.R;
+  if (writer && tid < E) {
+    const int r = tid / per_rank;
+    a.counts[tid] = t_e;
+    a.expert_off[tid] = r * a.region_rows + pre - s_pre[r * per_rank];
+  }
+  if (writer && tid == 0) a.expert_off[E] = a.R * a.region_rows;
   // pass 2: absolute bases of this thread's rows
   if (active) {
     const int rk = e / per_rank;
@@ -238,16 +237,21 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(RouteArgs a) {
   // ---- 2. arrival; the last P CTAs to arrive build the base table together
   const int P = min(G, kScanners);
   if (tid == 0) {
-    fence_acq_rel_gpu();  // this CTA's counts and totals before its arrival
+    // release: this CTA's counts and totals (ordered before by the block
+    // barrier) before its arrival
+    fence_acq_rel_gpu();
     const int arrival = int(atomicAdd(&ctrl->ticket, 1u));
     int ok = 1;
     if (arrival == G - 1) {
-      // every CTA has arrived: reset the counter, publish the new generation
+      // every CTA has arrived: reset the counter; the fence acquires every
+      // CTA's counts (this CTA scans too) and releases them with the new
+      // generation
       st_relaxed_gpu(&ctrl->ticket, 0u);
       fence_acq_rel_gpu();
       atomicAdd(&ctrl->rgen, 1u);
     } else if (arrival >= G - P) {
-      // a scanner: wait (bounded) until the last CTA has arrived
+      // a scanner: wait (bounded) until the last CTA has arrived; the
+      // acquiring load that sees the new generation orders the reads below
       const long long t0 = clock64();
       while (ld_acquire_gpu(&ctrl->rgen) == gen) {
         if (clock64() - t0 > (1ll << 31)) {
@@ -257,11 +261,15 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(RouteArgs a) {
         }
       }
     }
-    fence_acq_rel_gpu();  // every CTA's counts and totals before the reads below
+    // the other CTAs read nothing after their arrival
     s_arrival = arrival;
     s_ok = ok;
   }
   __syncthreads();
+  // Every CTA has started by now, so the next kernel in the stream may be
+  // scheduled behind the scanners; it still waits for this grid to finish
+  // before it reads anything.
+  grid_dependents_launch();
   const int arrival = s_arrival;
   if (arrival >= G - P && s_ok) {
     const int s_idx = arrival - (G - P);
@@ -269,7 +277,6 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(RouteArgs a) {
     scan_columns(a, tot, min(E, s_idx * per), min(E, (s_idx + 1) * per), s_idx == P - 1, s_part,
                  s_pre, s_wsum);
   }
-  grid_dependents_launch();
 }
 
 // One CTA per SM at most (a CTA of 1024 threads fills an SM): with more route
