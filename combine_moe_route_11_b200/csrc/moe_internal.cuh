@@ -186,18 +186,19 @@ __device__ __forceinline__ void fence_acq_rel_gpu() {
 }
 
 // Barrier across all `blocks` blocks of a grid whose blocks are all resident
-// (cooperative launch).  The block barrier orders the block's writes before
-// thread 0's release fence and arrival; the last arrival bumps the
+// (cooperative launch).  `gen` is the generation word as thread 0 read it
+// after the grid's dependency wait (no block of this grid can have bumped it
+// before this block arrives).  The block barrier orders the block's writes
+// before thread 0's release fence and arrival; the last arrival bumps the
 // generation, which the others poll with acquire loads.  The wait is bounded
 // (~2^31 cycles); on timeout it records MOE_ERR_TIMEOUT and returns false,
 // and the workspace must be re-initialised before its next use.
-__device__ __forceinline__ bool grid_barrier(void* ws, unsigned blocks) {
+__device__ __forceinline__ bool grid_barrier(void* ws, unsigned blocks, unsigned gen) {
   __shared__ int s_ok;
   Ctrl* c = reinterpret_cast<Ctrl*>(ws);
   __syncthreads();
   if (threadIdx.x == 0) {
     bool ok = true;
-    const unsigned gen = ld_acquire_gpu(&c->gen);
     fence_acq_rel_gpu();
     if (atomicAdd(&c->arrive, 1u) + 1u == blocks) {
       st_relaxed_gpu(&c->arrive, 0u);

@@ -52,7 +52,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_dispatch_kernel(FusedA
   extern __shared__ int32_t s_dyn[];  // masks [blocks, E], bases [blocks, E], picks [owned, K]
   __shared__ int32_t s_pre[kMaxExperts];
   __shared__ int32_t s_wsum[kWarps];
-  __shared__ unsigned s_parity;
+  __shared__ unsigned s_gen;
   const RouteArgs& a = f.r;
   const int E = a.E, K = a.K, B = a.blocks, n = a.n;
   const int G = gridDim.x;
@@ -65,7 +65,11 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_dispatch_kernel(FusedA
   const int mine = int(blockIdx.x) < n ? (n - 1 - int(blockIdx.x)) / G + 1 : 0;
   const int items = mine * f.chunks;  // (owned token i, chunk c) -> i * chunks + c
   grid_dependency_wait();
-  if (tid == 0) s_parity = ld_acquire_gpu(&reinterpret_cast<Ctrl*>(a.ws)->gen) & 1u;
+  unsigned gen = 0u;  // thread 0's copy of the barrier generation
+  if (tid == 0) {
+    gen = ld_acquire_gpu(&reinterpret_cast<Ctrl*>(a.ws)->gen);
+    s_gen = gen;
+  }
 
   // ---- the first chunk of x, in flight while routing runs
   uint4 v0 = make_uint4(0u, 0u, 0u, 0u);
@@ -75,7 +79,8 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_dispatch_kernel(FusedA
     if (g < f.vecs) v0 = ld_nc_v4(f.x + t * row_bytes + (g << 4));
   }
   __syncthreads();
-  uint32_t* gmask = a.masks + size_t(s_parity) * a.mask_rows * E;
+  const unsigned parity = s_gen & 1u;
+  uint32_t* gmask = a.masks + size_t(parity) * a.mask_rows * E;
 
   // ---- phase 1: one warp per owned token
   for (int i = warp; i < mine; i += kWarps) {
@@ -92,15 +97,22 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_dispatch_kernel(FusedA
     if (nonfinite && lane == 0) set_status(a.ws, MOE_ERR_NONFINITE);
   }
 
-  if (!grid_barrier(a.ws, G)) return;
+  if (!grid_barrier(a.ws, G, gen)) return;
 
   // ---- phase 2, in every block: masks, totals, offsets and the base table
   int tot = 0;
   if (tid < E) {
-    for (int b = 0; b < B; ++b) {
-      const uint32_t m = __ldcg(gmask + b * E + tid);
-      s_mask[b * E + tid] = m;
-      tot += __popc(m);
+    // eight rows' loads in flight at a time
+    for (int b0 = 0; b0 < B; b0 += 8) {
+      uint32_t m[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m[i] = b0 + i < B ? __ldcg(gmask + (b0 + i) * E + tid) : 0u;
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (b0 + i < B) {
+          s_mask[(b0 + i) * E + tid] = m[i];
+          tot += __popc(m[i]);
+        }
     }
   }
   int incl = tot;
@@ -140,7 +152,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_dispatch_kernel(FusedA
     }
   }
   if (blockIdx.x == 0) {
-    uint32_t* next = a.masks + size_t(s_parity ^ 1u) * a.mask_rows * E;
+    uint32_t* next = a.masks + size_t(parity ^ 1u) * a.mask_rows * E;
     for (int i = tid; i < a.mask_rows * E; i += kRouteThreads) next[i] = 0u;
     if (tid == 0) a.expert_off[E] = a.R * a.region_rows;
   }
