@@ -41,7 +41,7 @@ namespace moe {
 namespace {
 
 static_assert(kWarps == 32, "one warp per token of a 32-token route block");
-constexpr int kScanCache = 16;  // count-table rows a scanning thread keeps in registers
+constexpr int kScanCache = 8;   // count-table rows a scanning thread keeps in registers
 constexpr int kScanBatch = 8;  // count-table rows per batch when they are not all cached
 constexpr int kScanners = 8;   // CTAs that share the base table: the last ones to arrive
 
