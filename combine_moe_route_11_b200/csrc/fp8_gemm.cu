@@ -237,7 +237,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* pfull = empty + kStages;  // partial buffer b written by the MMAs
   uint64_t* pempty = pfull + 2;       // partial buffer b read by every promotion warp
   uint64_t* drained = pempty + 2;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drained + 1);
+  uint64_t* tq_full = drained + 1;
+  uint64_t* tq_empty = tq_full + kTileQ;
+  int* tq_slot = reinterpret_cast<int*>(tq_empty + kTileQ);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(tq_slot + kTileQ);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
   __shared__ int s_pref[kMaxExperts + 1];
   __shared__ int s_cnt[kMaxExperts];  // counts clamped to [0, T]
@@ -255,6 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&pempty[b], kPromoWarps);
     }
     mbar_init(drained, 1);
+    tq_init(TileQueue{tq_slot, tq_full, tq_empty, 0, 0u}, 1 + kPromoWarps);
     *s_abort = 0;
     fence_barrier_init();
   }
@@ -297,7 +301,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;  // copies issued, in ring order
-      for (int t = blockIdx.x; t < total && !*s_abort; t += gridDim.x) {
+      TileQueue q{tq_slot, tq_full, tq_empty, 0, 0u};
+      for (;;) {
+        // the next tile, published before its copies; `total` ends every loop
+        const int t = *s_abort ? total : tq_take(g.ws, total);
+        if (!tq_push(q, t)) {
+          set_status(g.ws, MOE_ERR_TIMEOUT);
+          *s_abort = 1;
+          break;
+        }
+        if (t >= total) break;
         const Tile tl = tile_of(t, s_pref, E, g.n_tiles);
         const int a_row = g.expert_off[tl.e] + tl.m * kBM;
         const int b_row = tl.e * g.b_rows + tl.n * (kSwiGLU ? kBN / 2 : kBN);
@@ -335,7 +348,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t phase = 0, buf_phase = 0;
     const uint32_t idesc = idesc_e4m3(kBN);
     bool ok = true;
-    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+    TileQueue q{tq_slot, tq_full, tq_empty, 0, 0u};
+    while (ok) {
+      int t = total;
+      bool got = true;
+      if (lane == 0) got = !*s_abort && tq_pop(q, &t);
+      got = __shfl_sync(0xFFFFFFFFu, got ? 1 : 0, 0) != 0;
+      t = __shfl_sync(0xFFFFFFFFu, t, 0);
+      if (!got) {
+        if (lane == 0 && !*s_abort) set_status(g.ws, MOE_ERR_TIMEOUT);
+        __syncwarp();
+        *s_abort = 1;
+        break;
+      }
+      if (t >= total) break;
       for (int kb = 0; kb < g.k_steps; ++kb) {
         bool w = !*s_abort;
         if (w) w = mbar_wait_hot(&full[stage], phase);
@@ -379,7 +405,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int b_blocks = g.b_rows / 128;    // weight-tile scale rows per expert
     int buf = 0;
     uint32_t buf_phase = 0;
-    for (int t = blockIdx.x; t < total && !*s_abort; t += gridDim.x) {
+    TileQueue q{tq_slot, tq_full, tq_empty, 0, 0u};
+    for (;;) {
+      int t = total;
+      bool got = true;
+      if (lane == 0) got = !*s_abort && tq_pop(q, &t);
+      got = __shfl_sync(0xFFFFFFFFu, got ? 1 : 0, 0) != 0;
+      t = __shfl_sync(0xFFFFFFFFu, t, 0);
+      if (!got) {
+        if (lane == 0 && !*s_abort) set_status(g.ws, MOE_ERR_TIMEOUT);
+        *s_abort = 1;
+        break;
+      }
+      if (t >= total) break;
       const Tile tl = tile_of(t, s_pref, E, g.n_tiles);
       const int rows = min(s_cnt[tl.e] - tl.m * kBM, kBM);
       const int64_t row = int64_t(g.expert_off[tl.e]) + tl.m * kBM + r_local;
@@ -466,6 +504,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
                  "r"(kTmemCols)
                  : "memory");
+  if (threadIdx.x == 0) tq_finish(g.ws);
   grid_dependents_launch();
 }
 

@@ -28,7 +28,9 @@ struct Ctrl {
   unsigned int gen;       // fused kernel's grid barrier: generation, bumped when all arrived
   unsigned int ticket;    // route kernel: route blocks arrived (reset by the last one)
   unsigned int rgen;      // route kernel: calls completed; selects the half of the totals
-  unsigned int pad[59];
+  unsigned int tile_next; // grouped GEMMs: next tile to hand out (reset by the last CTA)
+  unsigned int tile_done; // grouped GEMMs: CTAs finished (reset by the last one)
+  unsigned int pad[57];
 };
 static_assert(sizeof(Ctrl) == 256, "control block is 256 bytes");
 
@@ -281,6 +283,66 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   while (!mbar_try_wait(bar, parity))
     if (clock64() - t0 > (1ll << 31)) return false;
   return true;
+}
+
+// ---- dynamic tile scheduling for the persistent grouped GEMMs
+// Thread 0 of a CTA (the copy producer) takes tiles one at a time from a
+// counter in the workspace's control block, so a CTA that finishes early
+// takes more; it hands each index, in order, to the CTA's consumer warps
+// through a ring of kTileQ slots in shared memory (one mbarrier pair per
+// slot: `full` completes when the slot is written, `empty` when every
+// consumer warp has read it).  An index >= the tile count ends the loops.
+constexpr int kTileQ = 4;
+
+struct TileQueue {
+  int* slot;        // [kTileQ]
+  uint64_t* full;   // [kTileQ], one arrival (the producer)
+  uint64_t* empty;  // [kTileQ], one arrival per consumer warp
+  int i;
+  uint32_t phase;
+};
+
+__device__ __forceinline__ void tq_init(const TileQueue& q, uint32_t consumer_warps) {
+  for (int s = 0; s < kTileQ; ++s) {
+    mbar_init(&q.full[s], 1);
+    mbar_init(&q.empty[s], consumer_warps);
+  }
+}
+
+// Producer: publish tile t in the next slot; false if the wait gave up.
+__device__ __forceinline__ bool tq_push(TileQueue& q, int t) {
+  if (!mbar_wait(&q.empty[q.i], q.phase ^ 1u)) return false;
+  q.slot[q.i] = t;
+  mbar_arrive(&q.full[q.i]);
+  if (++q.i == kTileQ) q.i = 0, q.phase ^= 1u;
+  return true;
+}
+
+// One lane of a consumer warp: the next tile index, or false if the wait
+// gave up.  The slot is released as soon as it has been read.
+__device__ __forceinline__ bool tq_pop(TileQueue& q, int* t) {
+  if (!mbar_wait(&q.full[q.i], q.phase)) return false;
+  *t = q.slot[q.i];
+  mbar_arrive(&q.empty[q.i]);
+  if (++q.i == kTileQ) q.i = 0, q.phase ^= 1u;
+  return true;
+}
+
+// The next tile for this CTA (thread 0 only); `total` once all are taken.
+__device__ __forceinline__ int tq_take(void* ws, int total) {
+  const unsigned t = atomicAdd(&reinterpret_cast<Ctrl*>(ws)->tile_next, 1u);
+  return t < unsigned(total) ? int(t) : total;
+}
+
+// Thread 0 of every CTA, after its last access to the tile counter: the last
+// CTA of the grid to finish resets both counters for the next launch.
+__device__ __forceinline__ void tq_finish(void* ws) {
+  Ctrl* c = reinterpret_cast<Ctrl*>(ws);
+  fence_acq_rel_gpu();
+  if (atomicAdd(&c->tile_done, 1u) == gridDim.x - 1) {
+    atomicExch(&c->tile_next, 0u);
+    atomicExch(&c->tile_done, 0u);
+  }
 }
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }

@@ -175,7 +175,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* acc_full = empty + kStages;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drained = acc_empty + 2;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drained + 1);
+  uint64_t* tq_full = drained + 1;
+  uint64_t* tq_empty = tq_full + kTileQ;
+  int* tq_slot = reinterpret_cast<int*>(tq_empty + kTileQ);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(tq_slot + kTileQ);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
   __shared__ int s_pref[kMaxE + 1];
   __shared__ int s_cnt[kMaxE];  // counts clamped to [0, T]
@@ -193,6 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&acc_empty[b], kEpiWarps);
     }
     mbar_init(drained, 1);
+    tq_init(TileQueue{tq_slot, tq_full, tq_empty, 0, 0u}, 1 + kEpiWarps);
     *s_abort = 0;
     fence_barrier_init();
   }
@@ -237,7 +241,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t issued_phase[kStages];
       bool issued[kStages];
       for (int s = 0; s < kStages; ++s) issued[s] = false, issued_phase[s] = 0;
-      for (int t = blockIdx.x; t < total && !*s_abort; t += gridDim.x) {
+      TileQueue q{tq_slot, tq_full, tq_empty, 0, 0u};
+      for (;;) {
+        // the next tile, published before its copies; `total` ends every loop
+        const int t = *s_abort ? total : tq_take(g.ws, total);
+        if (!tq_push(q, t)) {
+          set_status(g.ws, MOE_ERR_TIMEOUT);
+          *s_abort = 1;
+          break;
+        }
+        if (t >= total) break;
         const Tile tl = tile_of(t, s_pref, E, g.n_tiles);
         const int a_row = g.expert_off[tl.e] + tl.m * kBM;
         const int b_row = tl.e * g.b_rows + tl.n * (kSwiGLU ? kBN / 2 : kBN);
@@ -271,7 +284,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
-      for (int t = blockIdx.x; t < total && !*s_abort; t += gridDim.x) {
+      TileQueue q{tq_slot, tq_full, tq_empty, 0, 0u};
+      for (;;) {
+        int t = total;
+        if (*s_abort || !tq_pop(q, &t)) {
+          if (!*s_abort) set_status(g.ws, MOE_ERR_TIMEOUT);
+          *s_abort = 1;
+          break;
+        }
+        if (t >= total) break;
         if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u)) {
           set_status(g.ws, MOE_ERR_TIMEOUT);
           *s_abort = 1;
@@ -327,7 +348,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r_local = quarter * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < total && !*s_abort; t += gridDim.x) {
+    TileQueue q{tq_slot, tq_full, tq_empty, 0, 0u};
+    for (;;) {
+      int t = total;
+      bool got = true;
+      if (lane == 0) got = !*s_abort && tq_pop(q, &t);
+      got = __shfl_sync(0xFFFFFFFFu, got ? 1 : 0, 0) != 0;
+      t = __shfl_sync(0xFFFFFFFFu, t, 0);
+      if (!got) {
+        if (lane == 0 && !*s_abort) set_status(g.ws, MOE_ERR_TIMEOUT);
+        *s_abort = 1;
+        break;
+      }
+      if (t >= total) break;
       const Tile tl = tile_of(t, s_pref, E, g.n_tiles);
       bool ready = true;
       if (lane == 0) ready = mbar_wait(&acc_full[acc], acc_phase);
@@ -439,6 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
                  "r"(kTmemCols)
                  : "memory");
+  if (threadIdx.x == 0) tq_finish(g.ws);
   grid_dependents_launch();
 }
 
