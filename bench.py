@@ -33,6 +33,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -117,13 +118,25 @@ def read_peaks() -> tuple[float, str]:
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def _strip_comments(code: bytes) -> bytes:
+    """C/C++ source without its comments and blank-line and trailing-space
+    differences: what the compiler sees of it (string literals in these
+    files hold no comment markers)."""
+    code = re.sub(rb"/\*.*?\*/", b" ", code, flags=re.S)
+    code = re.sub(rb"//[^\n]*", b"", code)
+    lines = [ln.rstrip() for ln in code.split(b"\n")]
+    return b"\n".join(ln for ln in lines if ln)
+
+
 def _device_part(name: str, start: bytes = b"", end: bytes = b"") -> bytes:
-    """The bytes of a source file between two markers (whole ends if absent)."""
+    """The code of a source file between two markers (whole ends if absent),
+    comments stripped, so that a record stays tied to the code it was taken
+    on and not to its comments."""
     with open(os.path.join(ROOT, "combine_moe_route_11_b200", "csrc", name), "rb") as f:
         text = f.read()
     a = text.find(start) if start and start in text else 0
     b = text.find(end) if end and end in text else len(text)
-    return text[a:b]
+    return _strip_comments(text[a:b])
 
 
 _HELPERS = b"// ------------------------------------------------------------------ device helpers"

@@ -33,7 +33,10 @@
 //               last k-block of a tile, SwiGLU (GEMM1) or conversion (GEMM2)
 //               and bf16 stores of the rows inside the expert's segment.
 // Tiles (expert, n-tile, m-tile) come from the routing counts with the m-tile
-// innermost, so the CTAs that share a weight tile run at the same time.
+// innermost; the producer thread takes them one at a time from a counter in
+// the workspace and hands each to the CTA's other warps, so a CTA that
+// finishes early takes more, and the CTAs that share a weight tile start it
+// at about the same time.
 // Every wait is bounded; on timeout the CTA records MOE_ERR_TIMEOUT, drains
 // its copies and MMAs, frees its tensor memory and returns.
 #include "moe_internal.cuh"

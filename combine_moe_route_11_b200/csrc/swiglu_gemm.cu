@@ -20,8 +20,10 @@
 //   warps 2..5  epilogue: tcgen05.ld of their 32-row quarter, SwiGLU (GEMM1)
 //               or conversion (GEMM2), bf16 stores of the valid rows.
 // Tiles (expert, n-tile, m-tile) are enumerated on the device from the
-// routing counts, m-tile innermost so the CTAs sharing a weight tile run at
-// the same time.  An expert's last m-tile usually holds only a few rows;
+// routing counts, m-tile innermost; the producer thread takes them one at a
+// time from a counter in the workspace and hands each to the CTA's other
+// warps, so a CTA that finishes early takes more, and the CTAs sharing a
+// weight tile start it at about the same time.  An expert's last m-tile usually holds only a few rows;
 // when it holds at most 96, the tile swaps the operand roles -- the weight
 // rows become the MMA's M side (two M=128 halves) and the token rows its N
 // side, rounded up to 16 -- so the tensor cores do work in proportion to
