@@ -164,3 +164,14 @@ def test_reference_line_reports_measured_steps(capsys):
     assert line["value"] == pytest.approx(line["tokens_per_step"] / (line["ms_per_step"] * 1e-3))
     assert line["cpu_baseline"]["cores"] >= 1 and "cpu_model" in line["cpu_baseline"]
     assert line["step_ms"]["n"] == 3
+
+
+def test_traffic_record_hash_ignores_comments_only():
+    """A traffic record stays tied to the code it was captured on: comment
+    edits keep the hash, a code edit changes it."""
+    import bench
+    a = b"// header\nint f(int x) {  /* twice */\n  return 2 * x;  // done\n}\n"
+    b = b"int f(int x) {\n\n  return 2 * x;\n}   \n// trailing note\n"
+    c = b"int f(int x) {\n  return 3 * x;\n}\n"
+    assert bench._strip_comments(a) == bench._strip_comments(b)
+    assert bench._strip_comments(a) != bench._strip_comments(c)
