@@ -25,7 +25,8 @@
 //   warp 1      owns the tensor memory (512 columns: two 128x256 fp32 partial
 //               buffers); one lane issues 4 x tcgen05.mma (M=128, N=256,
 //               K=32, e4m3 x e4m3 -> fp32) per k-block into the next free
-//               partial buffer and publishes it with tcgen05.commit;
+//               partial buffer and publishes it with one tcgen05.commit (the
+//               promotion warps free the stage when they see it);
 //   warps 2..9  two warps per 32-lane quarter of tensor memory, each keeping
 //               128 accumulator columns of its 32 rows in registers: wait for
 //               a partial buffer, tcgen05.ld, multiply by the row scale times
@@ -350,6 +351,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     int stage = 0, buf = 0;
     uint32_t phase = 0, buf_phase = 0;
     const uint32_t idesc = idesc_e4m3(kBN);
+    // descriptor of stage 0's A tile; a stage, the B tile and a K step are
+    // offsets in its 16-byte address field (shared addresses < 2^18)
+    const uint64_t desc0 = smem_desc_sw128(smem_addr(smem));
     bool ok = true;
     TileQueue q{tq_slot, tq_full, tq_empty, 0, 0u};
     while (ok) {
@@ -380,14 +384,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         if (lane == 0) {
           const uint32_t d_tmem = tmem_base + uint32_t(buf * kBN);
-          const uint32_t a_addr = smem_addr(smem + size_t(stage) * kStageBytes);
-          const uint32_t b_addr = a_addr + kABytes;
+          const uint64_t ad = desc0 + uint64_t((uint32_t(stage) * kStageBytes) >> 4);
+          const uint64_t bd = ad + uint64_t(kABytes >> 4);
 #pragma unroll
           for (int k = 0; k < kBK / kUmmaK; ++k)
-            umma_e4m3(d_tmem, smem_desc_sw128(a_addr + k * kUmmaK),
-                      smem_desc_sw128(b_addr + k * kUmmaK), idesc, k != 0 ? 1u : 0u);
-          umma_commit(&empty[stage]);  // stage free once these MMAs have read it
-          umma_commit(&pfull[buf]);    // partial sum of this k-block ready
+            umma_e4m3(d_tmem, ad + uint64_t(k * (kUmmaK >> 4)), bd + uint64_t(k * (kUmmaK >> 4)),
+                      idesc, k != 0 ? 1u : 0u);
+          // partial sum of this k-block ready; the promotion warps also free
+          // the stage when they see it (the MMAs have read it by then)
+          umma_commit(&pfull[buf]);
         }
         __syncwarp();
         if (++stage == kStages) stage = 0, phase ^= 1u;
@@ -406,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int half = (warp - 2) >> 2;       // which 128 of the tile's 256 columns
     const int r_local = quarter * 32 + lane;
     const int b_blocks = g.b_rows / 128;    // weight-tile scale rows per expert
-    int buf = 0;
+    int buf = 0, stage = 0;
     uint32_t buf_phase = 0;
     TileQueue q{tq_slot, tq_full, tq_empty, 0, 0u};
     for (;;) {
@@ -458,6 +463,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
+        if (warp == 2 && lane == 0) mbar_arrive(&empty[stage]);  // the stage's MMAs are done
+        if (++stage == kStages) stage = 0;
         const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(buf * kBN);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
