@@ -1,4 +1,5 @@
-"""Bounded device-side waits and CUDA-graph replays of the route kernel.
+"""Bounded device-side waits, and CUDA-graph replays of the kernels that keep
+state in the workspace's control block (route kernel, grouped GEMMs).
 
 The route kernel's scanners and the one-launch route + dispatch kernel's
 grid barrier wait on words in the workspace's control block.  Here the
@@ -140,4 +141,65 @@ def test_route_and_dispatch_replayed_in_a_cuda_graph(name, n):
         x_bits = parity.to_bits(inp["x"])
         tok = np.arange(slot_of.size) // cfg.top_k
         assert np.array_equal(recv[slot_of], x_bits[tok]), rep
+    del graph
+
+
+@pytest.mark.parametrize("fp8", [False, True], ids=["bf16_experts", "fp8_experts"])
+def test_layer_replayed_in_a_cuda_graph_equals_eager(fp8):
+    """The whole layer (route kernel, dispatch, grouped GEMMs with tiles taken
+    from the workspace counter, combine) captured once and replayed with
+    other inputs gives, on every replay, the bytes of an eager call on the
+    same inputs: the tile counter is reset by each launch's last CTA, and
+    which CTA computes a tile does not change its result.  1300 tokens take
+    the two-launch route + dispatch path; Zipf routing gives experts several
+    m-tiles."""
+    import combine_moe_route_11_b200 as mr
+    base = C["layer_fp8" if fp8 else "layer"]
+    cfg = base.replace(hidden=256, inter=256, n_experts=16, top_k=2, n_ranks=4, logits="zipf1.2")
+    n = 1300
+    dev = torch.device("cuda", 0)
+    plan = mr.Plan.from_config(cfg, n_max=n)
+    first = workloads.make_inputs(cfg, seed=90, n=n)
+    w = {k: first[k].to(dev) for k in ("w_gate_up", "w_gate_up_scale", "w_down", "w_down_scale")
+         if first.get(k) is not None}
+    logits = first["logits"].to(dev)
+    x = first["x"].to(dev)
+    xs = first["x_scale"].to(dev) if first.get("x_scale") is not None else None
+    out = torch.empty(n, cfg.hidden, dtype=torch.bfloat16, device=dev)
+    ws = plan.new_workspace(dev, layer=True)
+
+    def layer(stream=None):
+        if fp8:
+            mr.moe_layer_fp8(plan, logits, x, xs, w["w_gate_up"], w["w_gate_up_scale"],
+                             w["w_down"], w["w_down_scale"], out, ws, stream)
+        else:
+            mr.moe_layer(plan, logits, x, xs, w["w_gate_up"], w["w_down"], out, ws, stream)
+
+    def load(inp):
+        logits.copy_(inp["logits"].to(dev))
+        x.copy_(inp["x"].to(dev))
+        if xs is not None:
+            xs.copy_(inp["x_scale"].to(dev))
+
+    inputs = [workloads.make_inputs(cfg, seed=s, n=n) for s in (91, 92)]
+    eager = []
+    for inp in inputs:
+        load(inp)
+        layer()
+        assert mr.moe_get_status(plan, ws) == 0
+        eager.append(out.clone())
+    stream = torch.cuda.Stream(dev)
+    stream.wait_stream(torch.cuda.current_stream(dev))
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(graph, stream=stream):
+            layer(stream)
+    torch.cuda.current_stream(dev).wait_stream(stream)
+    for i in (0, 1, 0):
+        load(inputs[i])
+        torch.cuda.synchronize()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert mr.moe_get_status(plan, ws) == 0
+        assert torch.equal(out, eager[i]), f"replay of input {i} differs from the eager call"
     del graph
