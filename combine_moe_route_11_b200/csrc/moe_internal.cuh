@@ -26,11 +26,12 @@ struct Ctrl {
   unsigned int arrive;    // fused kernel's grid barrier: blocks arrived (reset by the last one)
   int status;             // first device-detected error, 0 = none
   unsigned int gen;       // fused kernel's grid barrier: generation, bumped when all arrived
-  unsigned int ticket;    // route kernel: route blocks arrived (reset by the last one)
-  unsigned int rgen;      // route kernel: calls completed; selects the half of the totals
+  unsigned int ticket;    // route kernel: CTAs arrived, calls of even generation
+  unsigned int rgen;      // route kernel: calls completed; selects counter and totals half
   unsigned int tile_next; // grouped GEMMs: next tile to hand out (reset by the last CTA)
   unsigned int tile_done; // grouped GEMMs: CTAs finished (reset by the last one)
-  unsigned int pad[57];
+  unsigned int ticket_b;  // route kernel: CTAs arrived, calls of odd generation
+  unsigned int pad[56];
 };
 static_assert(sizeof(Ctrl) == 256, "control block is 256 bytes");
 

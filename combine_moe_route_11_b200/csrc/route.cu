@@ -30,9 +30,10 @@
 //     Only CTAs that have finished their own blocks wait, at most P - 1 of
 //     them, so the others always have SMs to run on.
 // A slot is then base[block][e] + rank.  All integer results are
-// deterministic: no atomic decides an order.  The last arrival resets the
-// counter and bumps a generation word, which selects the half of the
-// double-buffered totals a call adds into (the previous call cleared it).
+// deterministic: no atomic decides an order.  A generation word, bumped by
+// each call's last arrival, selects which of two arrival counters and which
+// half of the double-buffered totals a call uses; CTA 0 clears the other
+// counter and half for the next call.
 #include "route_common.cuh"
 
 #include <type_traits>
@@ -185,8 +186,12 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(RouteArgs a) {
   __syncthreads();
   const unsigned gen = s_gen;
   int32_t* tot = a.totals + size_t(gen & 1u) * E;
-  if (blockIdx.x == 0)  // the other half starts the next call at zero
+  // this call's arrival counter; the other one starts the next call at zero
+  unsigned* ticket = (gen & 1u) ? &ctrl->ticket_b : &ctrl->ticket;
+  if (blockIdx.x == 0) {
     for (int i = tid; i < E; i += kRouteThreads) a.totals[size_t((gen & 1u) ^ 1u) * E + i] = 0;
+    if (tid == 0) st_relaxed_gpu((gen & 1u) ? &ctrl->ticket : &ctrl->ticket_b, 0u);
+  }
 
   for (int b = blockIdx.x; b < a.blocks; b += G) {
     const int t_base = b * kRouteTokens;
@@ -240,20 +245,18 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(RouteArgs a) {
     // release: this CTA's counts and totals (ordered before by the block
     // barrier) before its arrival
     fence_acq_rel_gpu();
-    const int arrival = int(atomicAdd(&ctrl->ticket, 1u));
+    const int arrival = int(atomicAdd(ticket, 1u));
     int ok = 1;
     if (arrival == G - 1) {
-      // every CTA has arrived: reset the counter; the fence acquires every
-      // CTA's counts (this CTA scans too) and releases them with the new
-      // generation
-      st_relaxed_gpu(&ctrl->ticket, 0u);
+      // every CTA has arrived: the fence acquires every CTA's counts (this
+      // CTA scans too); the next call uses the other counter and half
       fence_acq_rel_gpu();
       atomicAdd(&ctrl->rgen, 1u);
     } else if (arrival >= G - P) {
-      // a scanner: wait (bounded) until the last CTA has arrived; the
-      // acquiring load that sees the new generation orders the reads below
+      // a scanner: wait (bounded) until the counter shows every arrival; the
+      // acquiring load that sees it orders the reads below
       const long long t0 = clock64();
-      while (ld_acquire_gpu(&ctrl->rgen) == gen) {
+      while (ld_acquire_gpu(ticket) != unsigned(G)) {
         if (clock64() - t0 > (1ll << 31)) {
           set_status(a.ws, MOE_ERR_TIMEOUT);
           ok = 0;
