@@ -180,8 +180,8 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(RouteArgs a) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   Ctrl* ctrl = reinterpret_cast<Ctrl*>(a.ws);
   grid_dependency_wait();
-  // the generation of this call: it selects the half of the totals, and the
-  // last arrival bumps it once every CTA has read it
+  // the generation of this call: it selects the arrival counter and the half
+  // of the totals, and the last arrival bumps it once every CTA has read it
   if (tid == 0) s_gen = ld_acquire_gpu(&ctrl->rgen);
   __syncthreads();
   const unsigned gen = s_gen;
