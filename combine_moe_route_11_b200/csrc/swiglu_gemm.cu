@@ -240,9 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t issued_phase[kStages];
-      bool issued[kStages];
-      for (int s = 0; s < kStages; ++s) issued[s] = false, issued_phase[s] = 0;
+      int issued = 0;  // copies issued, in ring order
       TileQueue q{tq_slot, tq_full, tq_empty, 0, 0u};
       for (;;) {
         // the next tile, published before its copies; `total` ends every loop
@@ -272,14 +270,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             tma_load_2d(b_dst, &tma_b, kb * kBK, b_row, &full[stage]);
           }
-          issued[stage] = true;
-          issued_phase[stage] = phase;
+          ++issued;
           if (++stage == kStages) stage = 0, phase ^= 1u;
         }
       }
-      // never leave a copy in flight into this CTA's shared memory
-      for (int s = 0; s < kStages; ++s)
-        if (issued[s] && !mbar_wait(&full[s], issued_phase[s])) set_status(g.ws, MOE_ERR_TIMEOUT);
+      // never leave a copy in flight into this CTA's shared memory: a copy
+      // was only issued into a stage once the MMAs had consumed the copy
+      // before it, so only the last kStages copies can still be unwaited
+      for (int i = issued > kStages ? issued - kStages : 0; i < issued; ++i)
+        if (!mbar_wait(&full[i % kStages], uint32_t(i / kStages) & 1u))
+          set_status(g.ws, MOE_ERR_TIMEOUT);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
