@@ -101,6 +101,8 @@ CASES = [
     ("e48_k5", C["decode"].replace(n_experts=48, top_k=5, n_ranks=4, hidden=1024), 257, None),
     # 18 tiles, the last one ragged, over clusters of 4
     ("many_tiles_ragged", C["skewed"], 2300, None),
+    # 188 route blocks: the count kernel's CTAs take more than one each
+    ("route_blocks_per_cta", C["skewed"], 6001, np.arange(0, 6001, 7)),
     # k = 1 and k = E
     ("k1", C["decode"].replace(top_k=1, n_ranks=1), 130, None),
     ("k_eq_e", C["decode"].replace(n_experts=16, top_k=16, n_ranks=2, hidden=512), 70, None),

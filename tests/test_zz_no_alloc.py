@@ -47,7 +47,8 @@ def _route_noalloc(lib, plan, logits, out, stream):
                                       ctypes.c_void_p(stream.cuda_stream))
 
 
-@pytest.mark.parametrize("name,n", [("prefill", 4096), ("skewed", 3000), ("tiny", 61)])
+@pytest.mark.parametrize("name,n", [("prefill", 4096), ("skewed", 3000), ("skewed", 6001),
+                                    ("tiny", 61)])
 def test_noalloc_matches_workspace_route_twice(name, n):
     mr, lib = _lib()
     cfg = workloads.CONFIGS[name]
