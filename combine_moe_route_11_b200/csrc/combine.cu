@@ -88,6 +88,10 @@ __global__ void __launch_bounds__(kCThreads, 4) combine_kernel(CombineArgs a) {
   const int64_t n_items = int64_t(a.n) * a.chunks;
   const int64_t stride = int64_t(gridDim.x) * kCWarps;
   grid_dependency_wait();
+  // Every CTA that runs this line has started, so once all have, the next
+  // kernel in the stream may be scheduled into the SM room this grid leaves
+  // (it waits for this grid to finish before it reads anything).
+  grid_dependents_launch();
   for (int64_t item = int64_t(blockIdx.x) * kCWarps + (threadIdx.x >> 5); item < n_items;
        item += stride) {
     const int64_t t = item / a.chunks;
@@ -128,7 +132,6 @@ __global__ void __launch_bounds__(kCThreads, 4) combine_kernel(CombineArgs a) {
     }
     if (mine) store_out<TO, NE>(a.out + t * a.o_row_bytes + int64_t(g) * NE * sizeof(TO), acc);
   }
-  grid_dependents_launch();
 }
 
 template <typename TY, typename TO>

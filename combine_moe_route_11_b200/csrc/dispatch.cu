@@ -49,6 +49,10 @@ __global__ void __launch_bounds__(kThreads, 8) dispatch_kernel(DispatchArgs a) {
   const int64_t n_items = int64_t(a.n) * a.chunks;
   const int64_t stride = int64_t(gridDim.x) * kWarps;
   grid_dependency_wait();
+  // Every CTA that runs this line has started, so once all have, the next
+  // kernel in the stream may be scheduled into the SM room this grid leaves
+  // (it waits for this grid to finish before it reads anything).
+  grid_dependents_launch();
   for (int64_t item = int64_t(blockIdx.x) * kWarps + (threadIdx.x >> 5); item < n_items;
        item += stride) {
     const int64_t t = item / a.chunks;
@@ -108,7 +112,6 @@ __global__ void __launch_bounds__(kThreads, 8) dispatch_kernel(DispatchArgs a) {
       }
     }
   }
-  grid_dependents_launch();
 }
 
 }  // namespace
