@@ -139,11 +139,12 @@ MOE_API int64_t moe_recv_rows(const moe_plan* plan, int32_t n);
  * topk_w: device fp32 [n, k]; counts: device int32 [E]; expert_off: device
  * int32 [E + 1].  Also leaves in `ws` the per-block bases that moe_dispatch
  * uses for the slots of this routing.  n = 0 writes zero counts and offsets.
- * One launch: each block of 32 tokens routes them, writes its per-expert
- * counts and adds them into per-expert totals in `ws`; the last min(blocks,
- * 8) blocks to finish share the scan of all blocks' counts into the offsets
- * and per-block bases (each waits, bounded, only for the others to finish;
- * MOE_ERR_TIMEOUT in the status word if that wait ever ran out). */
+ * One launch of at most one CTA per SM: a CTA routes route blocks of 32
+ * tokens, writes each block's per-expert counts and adds them into
+ * per-expert totals in `ws`; the last min(CTAs, 8) CTAs to finish share the
+ * scan of all blocks' counts into the offsets and per-block bases (each
+ * waits, bounded, only for the others to finish; MOE_ERR_TIMEOUT in the
+ * status word if that wait ever ran out). */
 MOE_API moe_status moe_route_topk(const moe_plan* plan, int32_t n, const float* logits,
                           int32_t* topk_idx, float* topk_w, int32_t* counts,
                           int32_t* expert_off, void* ws, moe_stream_t stream);
